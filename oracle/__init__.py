@@ -1,0 +1,29 @@
+"""Oracle for the few-step Flash DiT hot path: a plain, slow fp64 CPU restatement.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or run
+anything in this package.  The product path (the ``few_step_dit_b200`` package
+and its CUDA library) never imports it, and this package never imports the
+product: the two share no code, headers, tables or helpers.
+
+Sources (web write-ups of arXiv 2609.15863, "LynnReal-Omni"):
+
+* [tokendh] tokendh.com news article on LynnReal-Omni, sections
+  "一个模型如何同时干七件事：原生多模态骨干网络" (backbone, token tags),
+  "训练的核心难题：怎么让模型又快又准" (flow matching, dual clocks, Flash
+  layer schedule and spatial token compression).
+* [PaperDaily] longzhangge PaperDaily, "LynnReal Lab视频恢复与生成：统一多模态控制，
+  Flash降至377毫秒", section 一 (input tags, control offset, dual clocks) and
+  section 二 "Flash怎么把22帧压到377毫秒" (compression, residual broadcast).
+
+Every floating-point step runs in float64.  Where the pages leave a step open
+the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
+
+Parity status per function: everything in ``dit.py`` is pinned by the CPU
+tests in ``tests/test_oracle_pins.py`` except the conventions that are pure
+definitions (weight init, time-embedding MLP, bias placement); those are
+"parity unpinned" in the sense that no page fixes them, so the GPU path is
+compared against this oracle's definition of them.
+"""
+
+from .dit import *  # noqa: F401,F403
