@@ -1,0 +1,256 @@
+"""Python API over the C ABI: torch tensors in, torch tensors out.
+
+PyTorch supplies device memory and streams only; every step runs in
+libfsdit.so.  Buffers (outputs, workspaces) are allocated here with torch, so
+the library itself allocates nothing.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+import torch
+
+from . import lib as L
+
+TORCH_OF = {L.F32: torch.float32, L.BF16: torch.bfloat16}
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def dtype_code(t_dtype):
+    return L.BF16 if t_dtype == torch.bfloat16 else L.F32
+
+
+def make_dims(hidden, heads, ffn, dtype, head_dim=128, rope_split=(32, 48, 48), rms_eps=1e-6,
+              rope_theta=10000.0):
+    d = L.Dims()
+    d.hidden, d.heads, d.head_dim, d.ffn = hidden, heads, head_dim, ffn
+    d.rope_split[:] = list(rope_split)
+    d.rms_eps, d.rope_theta = rms_eps, rope_theta
+    d.dtype = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return d
+
+
+def dims_of(w):
+    """Dims of a synthetic Workload."""
+    return make_dims(w.hidden, w.heads, w.ffn, L.F32 if w.dtype == "f32" else L.BF16,
+                     w.head_dim, w.rope_split, w.rms_eps, w.rope_theta)
+
+
+class BlockWeights:
+    """Device weights of one block (dict of tensors) and their C struct."""
+
+    def __init__(self, tensors: dict):
+        self.tensors = {k: v.contiguous() for k, v in tensors.items()}
+        self.struct = L.BlockWeights(*[self.tensors[k].data_ptr() for k in L.BLOCK_FIELDS])
+
+
+class IOWeights:
+    def __init__(self, tensors: dict):
+        self.tensors = {k: v.contiguous() for k, v in tensors.items()}
+        t = self.tensors
+        self.struct = L.IOWeights(*[t[k].data_ptr() for k in L.IO_FIELDS],
+                                  t["w_vin"].shape[1], t["w_tin"].shape[1], t["w_ain"].shape[1],
+                                  t["w_t1"].shape[1])
+
+
+def keep_map(T, H, W, device="cuda", stream=None):
+    """Device keep-index map of a T x H x W grid: (keep_idx, near_idx) int32."""
+    lib = L.load()
+    n_keep = lib.fsdit_keep_count(T, H, W)
+    keep_idx = torch.empty(max(n_keep, 1), dtype=torch.int32, device=device)
+    near_idx = torch.empty(max(T * H * W, 1), dtype=torch.int32, device=device)
+    L.call("fsdit_build_keep_map", T, H, W, L.ptr(keep_idx), L.ptr(near_idx), _stream(stream))
+    return keep_idx[:n_keep], near_idx[:T * H * W]
+
+
+class Sequence:
+    """Per-row tags of a packed sequence on the device, plus the keep map of
+    its target grid when `compress` is set."""
+
+    def __init__(self, tags: dict, grid, n_vrows, n_text, n_audio, device="cuda", compress=True,
+                 stream=None):
+        self.grid = tuple(grid)
+        self.n_vrows, self.n_text, self.n_audio = n_vrows, n_text, n_audio
+        self.n_tokens = n_vrows + n_text + n_audio
+        dev = torch.device(device)
+        self.pos = torch.as_tensor(np.ascontiguousarray(tags["pos"], np.int32)).to(dev)
+        self.modality = torch.as_tensor(np.ascontiguousarray(tags["modality"], np.uint8)).to(dev)
+        self.time_id = torch.as_tensor(np.ascontiguousarray(tags["time_id"], np.uint8)).to(dev)
+        self.out_mask = torch.as_tensor(np.ascontiguousarray(tags["out_mask"], np.uint8)).to(dev)
+        T, H, W = self.grid
+        self.n_grid = T * H * W
+        self.keep_idx = self.near_idx = None
+        self.n_keep = 0
+        if compress and self.n_grid > 0:
+            self.keep_idx, self.near_idx = keep_map(T, H, W, dev, stream)
+            self.n_keep = int(self.keep_idx.numel())
+        self.struct = self._make_struct(compress)
+        self.struct_full = self._make_struct(False)
+
+    @property
+    def n_compressed(self):
+        return self.n_keep + self.n_tokens - self.n_grid
+
+    def _make_struct(self, compress):
+        T, H, W = self.grid
+        s = L.Tokens()
+        s.n_tokens, s.n_vrows, s.n_text, s.n_audio = self.n_tokens, self.n_vrows, self.n_text, self.n_audio
+        s.grid_t, s.grid_h, s.grid_w = T, H, W
+        s.pos_thw = self.pos.data_ptr()
+        s.modality = self.modality.data_ptr()
+        s.time_id = self.time_id.data_ptr()
+        s.out_mask = self.out_mask.data_ptr()
+        if compress and self.keep_idx is not None:
+            s.keep_idx, s.n_keep, s.near_idx = self.keep_idx.data_ptr(), self.n_keep, self.near_idx.data_ptr()
+        else:
+            s.keep_idx, s.n_keep, s.near_idx = None, 0, None
+        return s
+
+    @classmethod
+    def from_workload(cls, w, tags, device="cuda", compress=None):
+        comp = any(w.compress) if compress is None else compress
+        return cls(tags, w.grid, w.n_video + w.n_control, w.n_text, w.n_audio, device, comp)
+
+
+# ---------------------------------------------------------------- single steps
+
+def gather_rows(x, pos, keep_idx, n_grid, stream=None):
+    n_rows, hidden = x.shape
+    n_keep = keep_idx.numel()
+    n_out = n_keep + n_rows - n_grid
+    xc = torch.empty(n_out, hidden, dtype=torch.float32, device=x.device)
+    posc = torch.empty(n_out, 3, dtype=torch.int32, device=x.device) if pos is not None else None
+    L.call("fsdit_gather_rows", L.ptr(x), L.ptr(pos), L.ptr(xc), L.ptr(posc), L.ptr(keep_idx),
+           n_keep, n_grid, n_rows, hidden, _stream(stream))
+    return xc, posc
+
+
+def broadcast_residual(x, yc, keep_idx, near_idx, n_grid, out=None, stream=None):
+    n_rows, hidden = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    L.call("fsdit_broadcast_residual", L.ptr(x), L.ptr(yc), L.ptr(out), L.ptr(keep_idx),
+           L.ptr(near_idx), keep_idx.numel(), n_grid, n_rows, hidden, _stream(stream))
+    return out
+
+
+def rmsnorm_cast(x, g, eps=1e-6, stream=None):
+    rows, hidden = x.shape
+    xn = torch.empty(rows, hidden, dtype=g.dtype, device=x.device)
+    L.call("fsdit_rmsnorm_cast", L.ptr(x), L.ptr(g), L.ptr(xn), rows, hidden, eps,
+           dtype_code(g.dtype), _stream(stream))
+    return xn
+
+
+def linear(dims, a, w, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, stream=None):
+    M, K = a.shape
+    N = w.shape[0]
+    if out is None:
+        od = torch.float32 if epilogue in (L.EPI_BIAS_F32, L.EPI_RESIDUAL) else a.dtype
+        out = torch.empty(M, N, dtype=od, device=a.device)
+    L.call("fsdit_linear", C.byref(dims), L.ptr(a), L.ptr(w), L.ptr(b), L.ptr(out), L.ptr(resid),
+           L.ptr(pos), M, N, K, epilogue, _stream(stream))
+    return out
+
+
+def attention(dims, qkv, out=None, stream=None):
+    n = qkv.shape[0]
+    if out is None:
+        out = torch.empty(n, dims.hidden, dtype=qkv.dtype, device=qkv.device)
+    L.call("fsdit_attention", C.byref(dims), L.ptr(qkv), L.ptr(out), n, _stream(stream))
+    return out
+
+
+def euler_step(x, v, row_modality, out_mask, t_cur, t_next, stream=None):
+    n_rows, width = x.shape
+    tc = (C.c_float * 4)(*[float(t) for t in t_cur])
+    tn = (C.c_float * 4)(*[float(t) for t in t_next])
+    L.call("flow_euler_step", L.ptr(x), L.ptr(v), L.ptr(row_modality), L.ptr(out_mask), n_rows, width,
+           tc, tn, _stream(stream))
+    return x
+
+
+def device_error(stream=None):
+    L.call("fsdit_device_error", _stream(stream))
+
+
+# ---------------------------------------------------------------- block / stack / sampler
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes, device):
+    """A cached uint8 device buffer of at least nbytes (caller-side allocation)."""
+    key = str(device)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        _ws_cache.pop(key, None)
+        buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def block_forward(dims, weights: BlockWeights, seq: Sequence, x_in, x_out=None, compress=True,
+                  stream=None):
+    lib = L.load()
+    tok = seq.struct if compress else seq.struct_full
+    nbytes = lib.fsdit_block_workspace_size(C.byref(dims), seq.n_tokens, tok.n_keep)
+    ws = workspace(nbytes, x_in.device)
+    if x_out is None:
+        x_out = torch.empty_like(x_in)
+    L.call("dit_block_forward", C.byref(dims), C.byref(weights.struct), C.byref(tok), L.ptr(x_in),
+           L.ptr(x_out), L.ptr(ws), ws.numel(), _stream(stream))
+    return x_out
+
+
+class Backbone:
+    """Stack of blocks + io weights, ready for dit_stack_forward / dit_flow_sample."""
+
+    def __init__(self, dims, layers, io: IOWeights, layer_compress):
+        self.dims = dims
+        self.layers = layers
+        self.io = io
+        n = len(layers)
+        self.n_layers = n
+        self.layer_structs = (L.BlockWeights * max(n, 1))(*[lw.struct for lw in layers])
+        self.compress = (C.c_uint8 * max(n, 1))(*[int(c) for c in layer_compress])
+
+    def workspace_bytes(self, seq: Sequence, compress=True, n_times=3):
+        tok = seq.struct if compress else seq.struct_full
+        return L.load().fsdit_stack_workspace_size(C.byref(self.dims), C.byref(self.io.struct),
+                                                   C.byref(tok), n_times)
+
+    def forward(self, seq: Sequence, time_table, video_lat, text_emb, audio_lat, compress=True,
+                v_video=None, v_audio=None, stream=None):
+        tok = seq.struct if compress else seq.struct_full
+        dev = video_lat.device
+        ws = workspace(self.workspace_bytes(seq, compress, len(time_table)), dev)
+        if v_video is None:
+            v_video = torch.empty(seq.n_vrows, self.io.struct.c_video, dtype=torch.float32, device=dev)
+        if v_audio is None:
+            v_audio = torch.empty(seq.n_audio, self.io.struct.c_audio, dtype=torch.float32, device=dev)
+        tt = (C.c_float * len(time_table))(*[float(t) for t in time_table])
+        L.call("dit_stack_forward", C.byref(self.dims), self.n_layers, self.layer_structs, self.compress,
+               C.byref(self.io.struct), C.byref(tok), tt, len(time_table), L.ptr(video_lat),
+               L.ptr(text_emb), L.ptr(audio_lat), L.ptr(v_video), L.ptr(v_audio), L.ptr(ws), ws.numel(),
+               _stream(stream))
+        return v_video, v_audio
+
+    def sample(self, seq: Sequence, video_clock, audio_clock, video_lat, text_emb, audio_lat,
+               compress=True, stream=None):
+        """Few-step sampler; updates video_lat / audio_lat in place and returns them."""
+        tok = seq.struct if compress else seq.struct_full
+        ws = workspace(self.workspace_bytes(seq, compress, 3), video_lat.device)
+        E = len(video_clock) - 1
+        tv = (C.c_float * (E + 1))(*[float(t) for t in video_clock])
+        ta = (C.c_float * (E + 1))(*[float(t) for t in audio_clock])
+        L.call("dit_flow_sample", C.byref(self.dims), self.n_layers, self.layer_structs, self.compress,
+               C.byref(self.io.struct), C.byref(tok), E, tv, ta, L.ptr(video_lat), L.ptr(text_emb),
+               L.ptr(audio_lat), L.ptr(ws), ws.numel(), _stream(stream))
+        return video_lat, audio_lat

@@ -1,0 +1,612 @@
+// C ABI of libfsdit: host-side argument checks, workspace layout and the
+// launch sequence of the block, the backbone stack and the sampler.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace fsdit {
+
+fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st);
+fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
+                           int n_keep, int n_grid, int n_rows, int hidden, cudaStream_t st);
+fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
+                              const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
+                              cudaStream_t st);
+fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
+                                 cudaStream_t st);
+fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
+                          const void* w_in, const void* b_in, const float* text_proj, const void* mod_emb,
+                          const float* temb, const uint8_t* modality, const uint8_t* time_id, int n_times, int ea,
+                          int eb, cudaStream_t st);
+fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, int t_freq, const void* w1,
+                             const void* b1, const void* w2, const void* b2, float* h1, float* temb, int hidden,
+                             cudaStream_t st);
+fsdit_status launch_heads(int dtype, const float* x, int row0, int rows, int hidden, const void* g, const void* w,
+                          const void* b, int C, float eps, float* out, cudaStream_t st);
+fsdit_status launch_euler(float* x, const float* v, const uint8_t* mod, const uint8_t* mask, int n_rows, int width,
+                          const float* t_cur, const float* t_next, cudaStream_t st);
+
+// ---------------------------------------------------------------- errors
+static thread_local char t_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+}
+
+fsdit_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return FSDIT_OK;
+  set_error("%s: %s", what, cudaGetErrorString(e));
+  return FSDIT_E_CUDA;
+}
+
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      n = v;
+    if (n <= 0) n = 148;
+  });
+  return n;
+}
+
+#define FS_TRY(expr)                        \
+  do {                                      \
+    fsdit_status _s = (expr);               \
+    if (_s != FSDIT_OK) return _s;          \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static fsdit_status need(const void* p, const char* name) {
+  if (p == nullptr) {
+    set_error("%s is NULL", name);
+    return FSDIT_E_NULL;
+  }
+  if (!aligned16(p)) {
+    set_error("%s is not 16-byte aligned", name);
+    return FSDIT_E_ALIGN;
+  }
+  return FSDIT_OK;
+}
+
+static size_t dsize(int dtype) { return dtype == FSDIT_BF16 ? 2 : 4; }
+
+static fsdit_status check_dims(const fsdit_dims* d) {
+  FS_TRY(need(d, "dims"));
+  if (d->dtype != FSDIT_F32 && d->dtype != FSDIT_BF16) {
+    set_error("dims.dtype %d is neither FSDIT_F32 nor FSDIT_BF16", d->dtype);
+    return FSDIT_E_DTYPE;
+  }
+  if (d->head_dim != 128 || d->heads <= 0 || d->hidden != d->heads * d->head_dim || d->hidden % 64 != 0 ||
+      d->hidden > 8192) {
+    set_error("dims: need head_dim 128, hidden = heads*128, hidden %% 64 == 0, hidden <= 8192 (got %d/%d/%d)",
+              d->hidden, d->heads, d->head_dim);
+    return FSDIT_E_SHAPE;
+  }
+  if (d->ffn <= 0 || d->ffn % 64 != 0) {
+    set_error("dims.ffn %d must be a positive multiple of 64", d->ffn);
+    return FSDIT_E_SHAPE;
+  }
+  const int* s = d->rope_split;
+  if (s[0] < 0 || s[1] < 0 || s[2] < 0 || (s[0] | s[1] | s[2]) & 1 || s[0] + s[1] + s[2] != d->head_dim) {
+    set_error("dims.rope_split must be three even widths summing to head_dim");
+    return FSDIT_E_SHAPE;
+  }
+  if (!(d->rms_eps >= 0.f) || !(d->rope_theta > 1.f)) {
+    set_error("dims: rms_eps must be >= 0 and rope_theta > 1");
+    return FSDIT_E_SHAPE;
+  }
+  return FSDIT_OK;
+}
+
+static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* out, int ldo, const float* resid,
+                         const int32_t* pos) {
+  EpiParams e;
+  e.epi = epi;
+  e.bias = bias;
+  e.out = out;
+  e.ldo = ldo;
+  e.resid = resid;
+  e.ldr = ldo;
+  e.pos = pos;
+  e.rope_cols = 2 * d->hidden;
+  e.head_dim = d->head_dim;
+  e.s0 = d->rope_split[0];
+  e.s1 = d->rope_split[1];
+  e.log2_theta = log2f(d->rope_theta);
+  return e;
+}
+
+fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep, int M, int N,
+                           int K, cudaStream_t st) {
+  if (M <= 0) return FSDIT_OK;
+  if (d->dtype == FSDIT_BF16) return launch_linear_tc(a, w, ep, M, N, K, st);
+  return launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
+}
+
+fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n, cudaStream_t st) {
+  if (n <= 0) return FSDIT_OK;
+  if (d->dtype == FSDIT_BF16) return launch_attention_tc(qkv, out, n, d->heads, d->hidden, st);
+  return launch_attention_simt(FSDIT_F32, qkv, out, n, d->heads, d->hidden, st);
+}
+
+// ---------------------------------------------------------------- workspace
+struct Carve {
+  uint8_t* base;
+  size_t off;
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  }
+};
+
+struct BlockWs {
+  float* xc;       // [n_c, hidden] compressed residual (compressed mode)
+  int32_t* posc;   // [n_c, 3]
+  void* xn;        // [n, hidden] GEMM operand (normalized x / attention output)
+  void* qkv;       // [n, 3 hidden]
+  void* u;         // [n, ffn]
+};
+
+static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, bool compressed) {
+  BlockWs w;
+  const int n = compressed ? n_c : n_rows;
+  w.xc = compressed ? (float*)c.take((size_t)n_c * d->hidden * 4) : nullptr;
+  w.posc = compressed ? (int32_t*)c.take((size_t)n_c * 3 * 4) : nullptr;
+  w.xn = c.take((size_t)n * d->hidden * dsize(d->dtype));
+  w.qkv = c.take((size_t)n * 3 * d->hidden * dsize(d->dtype));
+  w.u = c.take((size_t)n * d->ffn * dsize(d->dtype));
+  return w;
+}
+
+// ---------------------------------------------------------------- block body
+// x[n, hidden] (fp32, in place): x += attn(...); x += ffn(...).
+static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
+                               const int32_t* pos, int n, const BlockWs& ws, cudaStream_t st) {
+  const int H = d->hidden, F = d->ffn;
+  FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
+  FS_TRY(launch_linear(d, ws.xn, w->w_qkv, make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * H, nullptr, pos), n,
+                       3 * H, H, st));
+  FS_TRY(launch_attention(d, ws.qkv, ws.xn, n, st));
+  FS_TRY(launch_linear(d, ws.xn, w->w_o, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), n, H, H,
+                       st));
+  FS_TRY(launch_rmsnorm_cast(x_out, w->g_ffn, ws.xn, n, H, d->rms_eps, d->dtype, st));
+  FS_TRY(launch_linear(d, ws.xn, w->w_1, make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr), n, F, H, st));
+  FS_TRY(launch_linear(d, ws.u, w->w_2, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_2, x_out, H, x_out, nullptr), n, H, F,
+                       st));
+  return FSDIT_OK;
+}
+
+static fsdit_status check_block_weights(const fsdit_block_weights* w) {
+  FS_TRY(need(w, "weights"));
+  FS_TRY(need(w->w_qkv, "w_qkv"));
+  FS_TRY(need(w->b_qkv, "b_qkv"));
+  FS_TRY(need(w->w_o, "w_o"));
+  FS_TRY(need(w->b_o, "b_o"));
+  FS_TRY(need(w->w_1, "w_1"));
+  FS_TRY(need(w->b_1, "b_1"));
+  FS_TRY(need(w->w_2, "w_2"));
+  FS_TRY(need(w->b_2, "b_2"));
+  FS_TRY(need(w->g_attn, "g_attn"));
+  FS_TRY(need(w->g_ffn, "g_ffn"));
+  return FSDIT_OK;
+}
+
+static fsdit_status check_tokens(const fsdit_tokens* t, bool need_tags) {
+  FS_TRY(need(t, "tokens"));
+  if (t->n_tokens <= 0 || t->n_vrows < 0 || t->n_text < 0 || t->n_audio < 0 ||
+      t->n_vrows + t->n_text + t->n_audio != t->n_tokens) {
+    set_error("tokens: n_tokens (%d) must be n_vrows + n_text + n_audio (%d+%d+%d) and positive", t->n_tokens,
+              t->n_vrows, t->n_text, t->n_audio);
+    return FSDIT_E_SHAPE;
+  }
+  if (t->grid_t < 0 || t->grid_h < 0 || t->grid_w < 0 ||
+      (long long)t->grid_t * t->grid_h * t->grid_w > (long long)t->n_vrows) {
+    set_error("tokens: grid %dx%dx%d does not fit in the %d video rows", t->grid_t, t->grid_h, t->grid_w, t->n_vrows);
+    return FSDIT_E_SHAPE;
+  }
+  FS_TRY(need(t->pos_thw, "tokens.pos_thw"));
+  if (need_tags) {
+    if (t->modality == nullptr || t->time_id == nullptr || t->out_mask == nullptr) {
+      set_error("tokens: modality, time_id and out_mask are required");
+      return FSDIT_E_NULL;
+    }
+  }
+  if (t->keep_idx != nullptr) {
+    const int n_grid = t->grid_t * t->grid_h * t->grid_w;
+    if (n_grid <= 0 || t->near_idx == nullptr || t->n_keep != fsdit_keep_count(t->grid_t, t->grid_h, t->grid_w)) {
+      set_error("tokens: keep map needs a non-empty grid, near_idx and n_keep == %d (got %d)",
+                n_grid > 0 ? fsdit_keep_count(t->grid_t, t->grid_h, t->grid_w) : 0, t->n_keep);
+      return FSDIT_E_SHAPE;
+    }
+    if (!aligned16(t->keep_idx) || !aligned16(t->near_idx)) {
+      set_error("tokens: keep_idx / near_idx must be 16-byte aligned");
+      return FSDIT_E_ALIGN;
+    }
+  }
+  return FSDIT_OK;
+}
+
+static int n_compressed(const fsdit_tokens* t) {
+  const int n_grid = t->grid_t * t->grid_h * t->grid_w;
+  return t->n_keep + (t->n_tokens - n_grid);
+}
+
+}  // namespace fsdit
+
+using namespace fsdit;
+
+// ================================================================ C ABI
+
+extern "C" {
+
+const char* fsdit_last_error(void) { return t_err; }
+const char* fsdit_version(void) { return "fsdit 0.1 sm_100a"; }
+
+fsdit_status fsdit_device_error(fsdit_stream_t stream) {
+  FS_TRY(cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "cudaStreamSynchronize"));
+  int v = 0;
+  FS_TRY(cuda_check(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)), "read device error word"));
+  if (v != 0) {
+    int z = 0;
+    FS_TRY(cuda_check(cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)), "clear device error word"));
+    set_error("device error word 0x%x (%s%s)", v, (v & DEVERR_TIMEOUT) ? "bounded wait timed out " : "",
+              (v & DEVERR_TAGS) ? "row tags inconsistent with segments" : "");
+    return (v & DEVERR_TIMEOUT) ? FSDIT_E_TIMEOUT : FSDIT_E_SHAPE;
+  }
+  return FSDIT_OK;
+}
+
+int fsdit_keep_count(int T, int H, int W) {
+  if (T <= 0 || H <= 0 || W <= 0) return 0;
+  return T * (H / 2 + 1) * (W / 2 + 1);
+}
+
+size_t fsdit_block_workspace_size(const fsdit_dims* dims, int n_tokens, int n_keep) {
+  if (check_dims(dims) != FSDIT_OK || n_tokens <= 0) return 0;
+  Carve c{nullptr, 0};
+  // n_keep > 0 -> compressed; the compressed row count is bounded by n_tokens
+  carve_block(c, dims, n_tokens, n_tokens, n_keep > 0);
+  return c.off;
+}
+
+static size_t stack_carve(Carve& c, const fsdit_dims* d, const fsdit_io_weights* io, const fsdit_tokens* t,
+                          int n_times, float** x, float** temb, float** h1, float** tproj, float** vv, float** va,
+                          BlockWs* bw) {
+  const int N = t->n_tokens;
+  const bool comp = t->keep_idx != nullptr;
+  *x = (float*)c.take((size_t)N * d->hidden * 4);
+  *temb = (float*)c.take((size_t)n_times * d->hidden * 4);
+  *h1 = (float*)c.take((size_t)n_times * d->hidden * 4);
+  *tproj = (float*)c.take((size_t)(t->n_text > 0 ? t->n_text : 1) * d->hidden * 4);
+  *vv = (float*)c.take((size_t)(t->n_vrows > 0 ? t->n_vrows : 1) * io->c_video * 4);
+  *va = (float*)c.take((size_t)(t->n_audio > 0 ? t->n_audio : 1) * io->c_audio * 4);
+  // block buffers sized for the full sequence; the compressed residual needs n_c rows
+  const int n_c = comp ? n_compressed(t) : 0;
+  BlockWs w;
+  w.xc = comp ? (float*)c.take((size_t)n_c * d->hidden * 4) : nullptr;
+  w.posc = comp ? (int32_t*)c.take((size_t)n_c * 3 * 4) : nullptr;
+  w.xn = c.take((size_t)N * d->hidden * dsize(d->dtype));
+  w.qkv = c.take((size_t)N * 3 * d->hidden * dsize(d->dtype));
+  w.u = c.take((size_t)N * d->ffn * dsize(d->dtype));
+  *bw = w;
+  return c.off;
+}
+
+size_t fsdit_stack_workspace_size(const fsdit_dims* dims, const fsdit_io_weights* io, const fsdit_tokens* tok,
+                                  int n_times) {
+  if (check_dims(dims) != FSDIT_OK || io == nullptr || check_tokens(tok, false) != FSDIT_OK) return 0;
+  Carve c{nullptr, 0};
+  float *x, *temb, *h1, *tp, *vv, *va;
+  BlockWs bw;
+  return stack_carve(c, dims, io, tok, n_times > 0 ? n_times : 1, &x, &temb, &h1, &tp, &vv, &va, &bw);
+}
+
+fsdit_status fsdit_build_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, fsdit_stream_t stream) {
+  if (T <= 0 || H <= 0 || W <= 0) {
+    set_error("keep map: grid %dx%dx%d must be non-empty", T, H, W);
+    return FSDIT_E_SHAPE;
+  }
+  FS_TRY(need(keep_idx, "keep_idx"));
+  FS_TRY(need(near_idx, "near_idx"));
+  return launch_keep_map(T, H, W, keep_idx, near_idx, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, float* x_c, int32_t* pos_c, const int32_t* keep_idx,
+                               int n_keep, int n_grid, int n_rows, int hidden, fsdit_stream_t stream) {
+  FS_TRY(need(x, "x"));
+  FS_TRY(need(x_c, "x_c"));
+  FS_TRY(need(keep_idx, "keep_idx"));
+  if ((pos == nullptr) != (pos_c == nullptr)) {
+    set_error("pos and pos_c must both be given or both be NULL");
+    return FSDIT_E_NULL;
+  }
+  if (n_keep <= 0 || n_grid < n_keep || n_rows < n_grid || hidden <= 0 || hidden % 4 != 0) {
+    set_error("gather: need 0 < n_keep <= n_grid <= n_rows and hidden %% 4 == 0");
+    return FSDIT_E_SHAPE;
+  }
+  return launch_gather(x, pos, x_c, pos_c, keep_idx, n_keep, n_grid, n_rows, hidden, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_broadcast_residual(const float* x, const float* y_c, float* out, const int32_t* keep_idx,
+                                      const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
+                                      fsdit_stream_t stream) {
+  FS_TRY(need(x, "x"));
+  FS_TRY(need(y_c, "y_c"));
+  FS_TRY(need(out, "out"));
+  FS_TRY(need(keep_idx, "keep_idx"));
+  FS_TRY(need(near_idx, "near_idx"));
+  if (n_keep <= 0 || n_grid < n_keep || n_rows < n_grid || hidden <= 0 || hidden % 4 != 0) {
+    set_error("broadcast: need 0 < n_keep <= n_grid <= n_rows and hidden %% 4 == 0");
+    return FSDIT_E_SHAPE;
+  }
+  if (out == y_c) {
+    set_error("broadcast: out must not alias y_c");
+    return FSDIT_E_SHAPE;
+  }
+  return launch_broadcast(x, y_c, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
+                                fsdit_stream_t stream) {
+  FS_TRY(need(x, "x"));
+  FS_TRY(need(g, "g"));
+  FS_TRY(need(xn, "xn"));
+  if (dtype != FSDIT_F32 && dtype != FSDIT_BF16) {
+    set_error("rmsnorm_cast: bad dtype %d", dtype);
+    return FSDIT_E_DTYPE;
+  }
+  if (rows < 0 || hidden <= 0 || hidden % 8 != 0 || hidden > 8192) {
+    set_error("rmsnorm_cast: need hidden %% 8 == 0 and hidden <= 8192");
+    return FSDIT_E_SHAPE;
+  }
+  if (rows == 0) return FSDIT_OK;
+  return launch_rmsnorm_cast(x, g, xn, rows, hidden, eps, dtype, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, const void* b, void* out,
+                          const float* resid, const int32_t* pos, int M, int N, int K, int epilogue,
+                          fsdit_stream_t stream) {
+  FS_TRY(check_dims(dims));
+  FS_TRY(need(a, "a"));
+  FS_TRY(need(w, "w"));
+  FS_TRY(need(b, "b"));
+  FS_TRY(need(out, "out"));
+  if (M < 0 || N <= 0 || K <= 0 || K % 8 != 0 || N % 32 != 0) {
+    set_error("linear: need M >= 0, N %% 32 == 0, K %% 8 == 0 (got %d %d %d)", M, N, K);
+    return FSDIT_E_SHAPE;
+  }
+  if (epilogue < FSDIT_EPI_BIAS || epilogue > FSDIT_EPI_RESIDUAL) {
+    set_error("linear: unknown epilogue %d", epilogue);
+    return FSDIT_E_SHAPE;
+  }
+  if (epilogue == FSDIT_EPI_RESIDUAL) FS_TRY(need(resid, "resid"));
+  if (epilogue == FSDIT_EPI_QKV_ROPE) {
+    FS_TRY(need(pos, "pos"));
+    if (N != 3 * dims->hidden) {
+      set_error("linear: the RoPE epilogue needs N == 3*hidden");
+      return FSDIT_E_SHAPE;
+    }
+  }
+  EpiParams ep = make_ep(dims, epilogue, b, out, N, resid, pos);
+  return launch_linear(dims, a, w, ep, M, N, K, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n, fsdit_stream_t stream) {
+  FS_TRY(check_dims(dims));
+  FS_TRY(need(qkv, "qkv"));
+  FS_TRY(need(out, "out"));
+  if (n < 0) {
+    set_error("attention: n < 0");
+    return FSDIT_E_SHAPE;
+  }
+  return launch_attention(dims, qkv, out, n, (cudaStream_t)stream);
+}
+
+fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_block_weights* w, const fsdit_tokens* tok,
+                               const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
+                               fsdit_stream_t stream) {
+  FS_TRY(check_dims(dims));
+  FS_TRY(check_block_weights(w));
+  FS_TRY(check_tokens(tok, false));
+  FS_TRY(need(x_in, "x_in"));
+  FS_TRY(need(x_out, "x_out"));
+  FS_TRY(need(workspace, "workspace"));
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool comp = tok->keep_idx != nullptr;
+  const int n = tok->n_tokens;
+  const int n_grid = tok->grid_t * tok->grid_h * tok->grid_w;
+  const int n_c = comp ? n_compressed(tok) : n;
+  Carve c{(uint8_t*)workspace, 0};
+  BlockWs ws = carve_block(c, dims, n, n_c, comp);
+  if (c.off > ws_bytes) {
+    set_error("workspace: need %zu bytes, got %zu", c.off, ws_bytes);
+    return FSDIT_E_WORKSPACE;
+  }
+  if (!comp) return block_body(dims, w, const_cast<float*>(x_in), x_out, tok->pos_thw, n, ws, st);
+  FS_TRY(launch_gather(x_in, tok->pos_thw, ws.xc, ws.posc, tok->keep_idx, tok->n_keep, n_grid, n, dims->hidden, st));
+  FS_TRY(block_body(dims, w, ws.xc, ws.xc, ws.posc, n_c, ws, st));
+  if (x_out != x_in) {
+    FS_TRY(launch_broadcast(x_in, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, n, dims->hidden, st));
+  } else {
+    FS_TRY(launch_broadcast(x_out, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, n, dims->hidden,
+                            st));
+  }
+  return FSDIT_OK;
+}
+
+static fsdit_status check_io(const fsdit_dims* d, const fsdit_io_weights* io) {
+  FS_TRY(need(io, "io"));
+  const void* ptrs[] = {io->w_vin, io->b_vin, io->w_tin, io->b_tin, io->w_ain, io->b_ain, io->mod_emb, io->w_t1,
+                        io->b_t1,  io->w_t2,  io->b_t2,  io->g_out, io->w_vout, io->b_vout, io->w_aout, io->b_aout};
+  const char* names[] = {"w_vin", "b_vin", "w_tin", "b_tin", "w_ain", "b_ain", "mod_emb", "w_t1",
+                         "b_t1",  "w_t2",  "b_t2",  "g_out", "w_vout", "b_vout", "w_aout", "b_aout"};
+  for (int i = 0; i < 16; ++i) FS_TRY(need(ptrs[i], names[i]));
+  if (io->c_video <= 0 || io->c_video > 64 || io->c_audio <= 0 || io->c_audio > 64 || io->c_text <= 0 ||
+      io->c_text % 8 != 0 || io->t_freq <= 0 || io->t_freq % 2 != 0 || io->t_freq > 1024) {
+    set_error("io: need 0 < c_video, c_audio <= 64, c_text %% 8 == 0, even t_freq <= 1024");
+    return FSDIT_E_SHAPE;
+  }
+  (void)d;
+  return FSDIT_OK;
+}
+
+static fsdit_status stack_forward_impl(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
+                                       const uint8_t* layer_compress, const fsdit_io_weights* io,
+                                       const fsdit_tokens* tok, const float* time_table, int n_times,
+                                       const float* video_lat, const void* text_emb, const float* audio_lat,
+                                       float* v_video, float* v_audio, void* workspace, size_t ws_bytes,
+                                       cudaStream_t st) {
+  const int H = dims->hidden;
+  Carve c{(uint8_t*)workspace, 0};
+  float *x, *temb, *h1, *tproj, *vv_ws, *va_ws;
+  BlockWs bw;
+  stack_carve(c, dims, io, tok, n_times, &x, &temb, &h1, &tproj, &vv_ws, &va_ws, &bw);
+  if (c.off > ws_bytes) {
+    set_error("workspace: need %zu bytes, got %zu", c.off, ws_bytes);
+    return FSDIT_E_WORKSPACE;
+  }
+  // embedding
+  FS_TRY(launch_time_mlp(dims->dtype, time_table, n_times, io->t_freq, io->w_t1, io->b_t1, io->w_t2, io->b_t2, h1,
+                         temb, H, st));
+  if (tok->n_text > 0) {
+    EpiParams ep = make_ep(dims, FSDIT_EPI_BIAS_F32, io->b_tin, tproj, H, nullptr, nullptr);
+    FS_TRY(launch_linear(dims, text_emb, io->w_tin, ep, tok->n_text, H, io->c_text, st));
+  }
+  FS_TRY(launch_embed(dims->dtype, x, H, 0, tok->n_vrows, 1, video_lat, io->c_video, io->w_vin, io->b_vin, nullptr,
+                      io->mod_emb, temb, tok->modality, tok->time_id, n_times, FSDIT_MOD_VIDEO, FSDIT_MOD_CONTROL, st));
+  FS_TRY(launch_embed(dims->dtype, x, H, tok->n_vrows, tok->n_text, 0, nullptr, 0, nullptr, nullptr, tproj,
+                      io->mod_emb, temb, tok->modality, tok->time_id, n_times, FSDIT_MOD_TEXT, FSDIT_MOD_TEXT, st));
+  FS_TRY(launch_embed(dims->dtype, x, H, tok->n_vrows + tok->n_text, tok->n_audio, 1, audio_lat, io->c_audio,
+                      io->w_ain, io->b_ain, nullptr, io->mod_emb, temb, tok->modality, tok->time_id, n_times,
+                      FSDIT_MOD_AUDIO, FSDIT_MOD_AUDIO, st));
+  // layers; a run of compressed layers is one gather .. one broadcast
+  const int N = tok->n_tokens;
+  const int n_grid = tok->grid_t * tok->grid_h * tok->grid_w;
+  const int n_c = tok->keep_idx ? n_compressed(tok) : N;
+  int l = 0;
+  while (l < n_layers) {
+    if (!layer_compress[l] || tok->keep_idx == nullptr) {
+      FS_TRY(block_body(dims, &layers[l], x, x, tok->pos_thw, N, bw, st));
+      ++l;
+      continue;
+    }
+    FS_TRY(launch_gather(x, tok->pos_thw, bw.xc, bw.posc, tok->keep_idx, tok->n_keep, n_grid, N, H, st));
+    while (l < n_layers && layer_compress[l]) {
+      FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, n_c, bw, st));
+      ++l;
+    }
+    FS_TRY(launch_broadcast(x, bw.xc, x, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, N, H, st));
+  }
+  // heads
+  FS_TRY(launch_heads(dims->dtype, x, 0, tok->n_vrows, H, io->g_out, io->w_vout, io->b_vout, io->c_video,
+                      dims->rms_eps, v_video, st));
+  FS_TRY(launch_heads(dims->dtype, x, tok->n_vrows + tok->n_text, tok->n_audio, H, io->g_out, io->w_aout, io->b_aout,
+                      io->c_audio, dims->rms_eps, v_audio, st));
+  return FSDIT_OK;
+}
+
+static fsdit_status check_stack_args(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
+                                     const uint8_t* layer_compress, const fsdit_io_weights* io,
+                                     const fsdit_tokens* tok, int n_times, const float* video_lat,
+                                     const void* text_emb, const float* audio_lat, const void* workspace) {
+  FS_TRY(check_dims(dims));
+  FS_TRY(check_io(dims, io));
+  FS_TRY(check_tokens(tok, true));
+  if (n_layers < 0 || (n_layers > 0 && (layers == nullptr || layer_compress == nullptr))) {
+    set_error("stack: n_layers >= 0 and host arrays layers / layer_compress are required");
+    return FSDIT_E_NULL;
+  }
+  for (int l = 0; l < n_layers; ++l) FS_TRY(check_block_weights(&layers[l]));
+  if (n_times <= 0 || n_times > 8) {
+    set_error("stack: 1 <= n_times <= 8");
+    return FSDIT_E_SHAPE;
+  }
+  if (tok->n_vrows > 0) FS_TRY(need(video_lat, "video_lat"));
+  if (tok->n_text > 0) FS_TRY(need(text_emb, "text_emb"));
+  if (tok->n_audio > 0) FS_TRY(need(audio_lat, "audio_lat"));
+  FS_TRY(need(workspace, "workspace"));
+  return FSDIT_OK;
+}
+
+fsdit_status dit_stack_forward(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
+                               const uint8_t* layer_compress, const fsdit_io_weights* io, const fsdit_tokens* tok,
+                               const float* time_table, int n_times, const float* video_lat, const void* text_emb,
+                               const float* audio_lat, float* v_video, float* v_audio, void* workspace,
+                               size_t ws_bytes, fsdit_stream_t stream) {
+  FS_TRY(check_stack_args(dims, n_layers, layers, layer_compress, io, tok, n_times, video_lat, text_emb, audio_lat,
+                          workspace));
+  if (time_table == nullptr) {
+    set_error("time_table is NULL");
+    return FSDIT_E_NULL;
+  }
+  if (tok->n_vrows > 0) FS_TRY(need(v_video, "v_video"));
+  if (tok->n_audio > 0) FS_TRY(need(v_audio, "v_audio"));
+  return stack_forward_impl(dims, n_layers, layers, layer_compress, io, tok, time_table, n_times, video_lat, text_emb,
+                            audio_lat, v_video, v_audio, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+fsdit_status flow_euler_step(float* x, const float* v, const uint8_t* row_modality, const uint8_t* out_mask,
+                             int n_rows, int row_width, const float* t_cur, const float* t_next,
+                             fsdit_stream_t stream) {
+  if (n_rows < 0 || row_width <= 0) {
+    set_error("euler: need n_rows >= 0 and row_width > 0");
+    return FSDIT_E_SHAPE;
+  }
+  if (n_rows == 0) return FSDIT_OK;
+  FS_TRY(need(x, "x"));
+  FS_TRY(need(v, "v"));
+  if (row_modality == nullptr || out_mask == nullptr || t_cur == nullptr || t_next == nullptr) {
+    set_error("euler: row_modality, out_mask, t_cur and t_next are required");
+    return FSDIT_E_NULL;
+  }
+  return launch_euler(x, v, row_modality, out_mask, n_rows, row_width, t_cur, t_next, (cudaStream_t)stream);
+}
+
+fsdit_status dit_flow_sample(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
+                             const uint8_t* layer_compress, const fsdit_io_weights* io, const fsdit_tokens* tok,
+                             int n_evals, const float* t_video, const float* t_audio, float* video_lat,
+                             const void* text_emb, float* audio_lat, void* workspace, size_t ws_bytes,
+                             fsdit_stream_t stream) {
+  FS_TRY(check_stack_args(dims, n_layers, layers, layer_compress, io, tok, 3, video_lat, text_emb, audio_lat,
+                          workspace));
+  if (n_evals <= 0 || t_video == nullptr || t_audio == nullptr) {
+    set_error("sample: n_evals > 0 and host clocks t_video / t_audio [n_evals+1] are required");
+    return FSDIT_E_SHAPE;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  Carve c{(uint8_t*)workspace, 0};
+  float *x, *temb, *h1, *tproj, *vv, *va;
+  BlockWs bw;
+  stack_carve(c, dims, io, tok, 3, &x, &temb, &h1, &tproj, &vv, &va, &bw);
+  if (c.off > ws_bytes) {
+    set_error("workspace: need %zu bytes, got %zu", c.off, ws_bytes);
+    return FSDIT_E_WORKSPACE;
+  }
+  const uint8_t* vid_mod = tok->modality;
+  const uint8_t* vid_mask = tok->out_mask;
+  const uint8_t* aud_mod = tok->modality + tok->n_vrows + tok->n_text;
+  const uint8_t* aud_mask = tok->out_mask + tok->n_vrows + tok->n_text;
+  for (int e = 0; e < n_evals; ++e) {
+    const float table[3] = {0.0f, t_video[e], t_audio[e]};
+    FS_TRY(stack_forward_impl(dims, n_layers, layers, layer_compress, io, tok, table, 3, video_lat, text_emb,
+                              audio_lat, vv, va, workspace, ws_bytes, st));
+    const float tc[4] = {0.0f, t_video[e], t_audio[e], 0.0f};
+    const float tn[4] = {0.0f, t_video[e + 1], t_audio[e + 1], 0.0f};
+    if (tok->n_vrows > 0) FS_TRY(launch_euler(video_lat, vv, vid_mod, vid_mask, tok->n_vrows, io->c_video, tc, tn, st));
+    if (tok->n_audio > 0) FS_TRY(launch_euler(audio_lat, va, aud_mod, aud_mask, tok->n_audio, io->c_audio, tc, tn, st));
+  }
+  return FSDIT_OK;
+}
+
+}  // extern "C"

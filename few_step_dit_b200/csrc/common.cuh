@@ -1,0 +1,157 @@
+// Shared device helpers of libfsdit (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fsdit.h"
+
+namespace fsdit {
+
+typedef __nv_bfloat16 bf16;
+
+// Device error word: kernels that give up a bounded wait set it; the host
+// reads it through fsdit_device_error().
+__device__ int g_device_error = 0;  // one translation unit (libfsdit.cu) includes every source
+
+enum { DEVERR_TIMEOUT = 1, DEVERR_TAGS = 2 };
+
+__device__ __forceinline__ void raise_device_error(int code) { atomicOr(&g_device_error, code); }
+
+template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
+template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }
+template <> __device__ __forceinline__ float ld_f32<bf16>(const bf16* p) { return __bfloat162float(*p); }
+
+template <typename T> __device__ __forceinline__ T cvt_from_f32(float v);
+template <> __device__ __forceinline__ float cvt_from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 cvt_from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  const float k1 = 0.044715f;
+  return 0.5f * x * (1.0f + tanhf(k0 * (x + k1 * x * x * x)));
+}
+
+// 3D RoPE rotation of one interleaved pair.  `d` is the even channel index of
+// the pair inside its head; the head is cut into chunks of s0 (t), s1 (h) and
+// the rest (w) channels; inside chunk a (width da, pair jj) the pair turns by
+// pos_a * theta^(-2 jj / da).
+__device__ __forceinline__ void rope_pair(float& a, float& b, int d, int s0, int s1, int head_dim,
+                                          const int32_t* pos3, float log2_theta) {
+  int axis, off, da;
+  if (d < s0) { axis = 0; off = 0; da = s0; }
+  else if (d < s0 + s1) { axis = 1; off = s0; da = s1; }
+  else { axis = 2; off = s0 + s1; da = head_dim - s0 - s1; }
+  const float jj = (float)((d - off) >> 1);
+  const float inv_freq = exp2f(-(2.0f * jj / (float)da) * log2_theta);
+  const float ang = (float)pos3[axis] * inv_freq;
+  float s, c;
+  sincosf(ang, &s, &c);
+  const float na = a * c - b * s;
+  const float nb = a * s + b * c;
+  a = na;
+  b = nb;
+}
+
+struct EpiParams {
+  int epi;              // FSDIT_EPI_*
+  const void* bias;     // [N], weight dtype
+  void* out;            // [M, ldo]
+  int ldo;
+  const float* resid;   // [M, ldr] (FSDIT_EPI_RESIDUAL)
+  int ldr;
+  const int32_t* pos;   // [M][3] (FSDIT_EPI_QKV_ROPE)
+  int rope_cols;        // columns [0, rope_cols) are rotated
+  int head_dim, s0, s1;
+  float log2_theta;
+};
+
+// Apply the epilogue to `cnt` consecutive columns [col, col+cnt) of one row.
+// v[] holds the fp32 accumulators; cnt is even and col is even.
+template <typename TW, int CNT>
+__device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int col, float* v) {
+  const TW* bias = reinterpret_cast<const TW*>(p.bias);
+#pragma unroll
+  for (int i = 0; i < CNT; ++i) v[i] += ld_f32<TW>(bias + col + i);
+  if (p.epi == FSDIT_EPI_QKV_ROPE) {
+    if (col < p.rope_cols) {
+      const int32_t* pos3 = p.pos + (size_t)row * 3;
+#pragma unroll
+      for (int i = 0; i < CNT; i += 2) {
+        int d = (col + i) % p.head_dim;
+        rope_pair(v[i], v[i + 1], d, p.s0, p.s1, p.head_dim, pos3, p.log2_theta);
+      }
+    }
+  } else if (p.epi == FSDIT_EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < CNT; ++i) v[i] = gelu_tanh(v[i]);
+  }
+  if (p.epi == FSDIT_EPI_RESIDUAL) {
+    const float* r = p.resid + (size_t)row * p.ldr + col;
+    float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
+    if constexpr (CNT % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < CNT; i += 4) {
+        float4 rv = *reinterpret_cast<const float4*>(r + i);
+        float4 ov = make_float4(rv.x + v[i], rv.y + v[i + 1], rv.z + v[i + 2], rv.w + v[i + 3]);
+        *reinterpret_cast<float4*>(o + i) = ov;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < CNT; ++i) o[i] = r[i] + v[i];
+    }
+  } else if (p.epi == FSDIT_EPI_BIAS_F32) {
+    float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
+    if constexpr (CNT % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < CNT; i += 4)
+        *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CNT; ++i) o[i] = v[i];
+    }
+  } else {
+    TW* o = reinterpret_cast<TW*>(p.out) + (size_t)row * p.ldo + col;
+    if constexpr (sizeof(TW) == 2 && CNT % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < CNT; i += 8) {
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i], v[i + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[i + 2], v[i + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[i + 4], v[i + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[i + 6], v[i + 7]);
+        uint4 u;
+        u.x = *reinterpret_cast<uint32_t*>(&h0);
+        u.y = *reinterpret_cast<uint32_t*>(&h1);
+        u.z = *reinterpret_cast<uint32_t*>(&h2);
+        u.w = *reinterpret_cast<uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(o + i) = u;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < CNT; ++i) o[i] = cvt_from_f32<TW>(v[i]);
+    }
+  }
+}
+
+}  // namespace fsdit
+
+// Host-side internal API shared by the .cu files.
+namespace fsdit {
+int num_sms();
+void set_error(const char* fmt, ...);
+fsdit_status cuda_check(cudaError_t e, const char* what);
+
+fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep,
+                           int M, int N, int K, cudaStream_t st);
+fsdit_status launch_linear_simt(int dtype, const void* a, const void* w, const EpiParams& ep,
+                                int M, int N, int K, cudaStream_t st);
+fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep, int M, int N,
+                              int K, cudaStream_t st);
+fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n,
+                              cudaStream_t st);
+fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n, int heads,
+                                   int hidden, cudaStream_t st);
+fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int hidden,
+                                 cudaStream_t st);
+}  // namespace fsdit

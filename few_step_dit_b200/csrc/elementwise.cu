@@ -1,0 +1,472 @@
+// HBM-bound kernels of the hot path: keep-index map, gather, nearest-kept
+// broadcast + residual, RMSNorm-cast, embedding, timestep MLP, output heads
+// and the per-modality Euler step.  All rows are moved with 16-byte vector
+// accesses; grids are sized from the SM count.
+#include "common.cuh"
+
+namespace fsdit {
+
+
+// ---------------------------------------------------------------- keep map
+
+// kept count of one axis of length n: floor(n/2) + 1
+__device__ __forceinline__ int axis_kept(int n) { return n / 2 + 1; }
+// nearest kept index (ties -> lower): i itself if even or last, else i-1
+__device__ __forceinline__ int axis_rho(int i, int n) { return ((i & 1) == 0 || i == n - 1) ? i : i - 1; }
+// compact index of a kept index i
+__device__ __forceinline__ int axis_kappa(int i) { return (i + 1) >> 1; }
+
+__global__ void keep_map_kernel(int T, int H, int W, int32_t* __restrict__ keep_idx,
+                                int32_t* __restrict__ near_idx) {
+  const int total = T * H * W;
+  const int kh = axis_kept(H), kw = axis_kept(W);
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < total; p += gridDim.x * blockDim.x) {
+    const int t = p / (H * W);
+    const int h = (p / W) % H;
+    const int w = p % W;
+    const int rh = axis_rho(h, H), rw = axis_rho(w, W);
+    const int c = t * kh * kw + axis_kappa(rh) * kw + axis_kappa(rw);
+    near_idx[p] = c;
+    if (rh == h && rw == w) keep_idx[c] = p;
+  }
+}
+
+// ---------------------------------------------------------------- gather
+
+// One block per output row (grid-stride over rows); float4 copies.
+__global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* __restrict__ pos,
+                                   float* __restrict__ xc, int32_t* __restrict__ posc,
+                                   const int32_t* __restrict__ keep_idx, int n_keep, int n_grid,
+                                   int n_out, int hidden) {
+  const int h4 = hidden >> 2;
+  for (int r = blockIdx.x; r < n_out; r += gridDim.x) {
+    const int src = r < n_keep ? keep_idx[r] : n_grid + (r - n_keep);
+    const float4* s = reinterpret_cast<const float4*>(x + (size_t)src * hidden);
+    float4* d = reinterpret_cast<float4*>(xc + (size_t)r * hidden);
+    for (int i = threadIdx.x; i < h4; i += blockDim.x) d[i] = __ldg(s + i);
+    if (pos != nullptr && threadIdx.x < 3) posc[(size_t)r * 3 + threadIdx.x] = pos[(size_t)src * 3 + threadIdx.x];
+  }
+}
+
+// ---------------------------------------------------------------- broadcast
+// phase 0: every row (out != x); phase 1: dropped grid rows only; phase 2:
+// kept grid rows and non-grid rows (phases 1 then 2 make the in-place form).
+__global__ void broadcast_kernel(const float* __restrict__ x, const float* __restrict__ yc,
+                                 float* __restrict__ out, const int32_t* __restrict__ keep_idx,
+                                 const int32_t* __restrict__ near_idx, int n_keep, int n_grid,
+                                 int n_rows, int hidden, int phase) {
+  const int h4 = hidden >> 2;
+  for (int p = blockIdx.x; p < n_rows; p += gridDim.x) {
+    float4* o = reinterpret_cast<float4*>(out + (size_t)p * hidden);
+    if (p < n_grid) {
+      const int c = near_idx[p];
+      const int src = keep_idx[c];
+      const float4* y = reinterpret_cast<const float4*>(yc + (size_t)c * hidden);
+      if (src == p) {
+        if (phase == 1) continue;
+        for (int i = threadIdx.x; i < h4; i += blockDim.x) o[i] = __ldg(y + i);
+      } else {
+        if (phase == 2) continue;
+        const float4* xp = reinterpret_cast<const float4*>(x + (size_t)p * hidden);
+        const float4* xk = reinterpret_cast<const float4*>(x + (size_t)src * hidden);
+        for (int i = threadIdx.x; i < h4; i += blockDim.x) {
+          const float4 a = xp[i], b = __ldg(y + i), k = xk[i];
+          o[i] = make_float4(a.x + (b.x - k.x), a.y + (b.y - k.y), a.z + (b.z - k.z), a.w + (b.w - k.w));
+        }
+      }
+    } else {
+      if (phase == 1) continue;
+      const float4* y = reinterpret_cast<const float4*>(yc + (size_t)(n_keep + p - n_grid) * hidden);
+      for (int i = threadIdx.x; i < h4; i += blockDim.x) o[i] = __ldg(y + i);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- RMSNorm-cast
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  const int nw = blockDim.x >> 5;
+  for (int i = 0; i < nw; ++i) s += red[i];
+  return s;
+}
+
+template <typename TO, typename TG>
+__device__ __forceinline__ void store4(TO* o, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float, float>(float* o, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(o) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16, bf16>(bf16* o, float a, float b, float c, float d) {
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(a, b), h1 = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&h0);
+  u.y = *reinterpret_cast<uint32_t*>(&h1);
+  *reinterpret_cast<uint2*>(o) = u;
+}
+
+template <typename T>
+__device__ __forceinline__ float4 load_g4(const T* g);
+template <>
+__device__ __forceinline__ float4 load_g4<float>(const float* g) { return __ldg(reinterpret_cast<const float4*>(g)); }
+template <>
+__device__ __forceinline__ float4 load_g4<bf16>(const bf16* g) {
+  uint2 u = __ldg(reinterpret_cast<const uint2*>(g));
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x), b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// One block (256 threads) per row; the row stays in registers between the
+// sum-of-squares pass and the scaled store.  hidden <= 256*4*RMS_MAXV.
+constexpr int RMS_MAXV = 8;
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_cast_kernel(const float* __restrict__ x, const T* __restrict__ g,
+                                                           T* __restrict__ xn, int rows, int hidden, float eps) {
+  __shared__ float red[32];
+  const int h4 = hidden >> 2;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * hidden);
+    float4 v[RMS_MAXV];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < RMS_MAXV; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      if (i < h4) {
+        v[k] = xr[i];
+        ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+      }
+    }
+    const float tot = block_sum(ss, red);
+    const float rstd = rsqrtf(tot / (float)hidden + eps);
+    T* o = xn + (size_t)r * hidden;
+#pragma unroll
+    for (int k = 0; k < RMS_MAXV; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      if (i < h4) {
+        const float4 gg = load_g4<T>(g + 4 * i);
+        store4<T, T>(o + 4 * i, v[k].x * rstd * gg.x, v[k].y * rstd * gg.y, v[k].z * rstd * gg.z,
+                     v[k].w * rstd * gg.w);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- embedding
+// x[r] = src(r) + mod_emb[modality[r]] + temb[time_id[r]], where src(r) is the
+// small-K projection lat[r'] W^T + b of a video/control or audio row, or the
+// precomputed text projection row.  A block owns EMB_ROWS consecutive rows of
+// one segment; each thread keeps one W row in registers and reuses it across
+// the block's rows.
+constexpr int EMB_ROWS = 16;
+constexpr int EMB_MAXK = 64;
+
+template <typename TW>
+__global__ void __launch_bounds__(256) embed_kernel(
+    float* __restrict__ x, int hidden, int row0, int rows, int kind,  // kind: 0 text, 1 latent
+    const float* __restrict__ lat, int K, const TW* __restrict__ w_in, const TW* __restrict__ b_in,
+    const float* __restrict__ text_proj, const TW* __restrict__ mod_emb, const float* __restrict__ temb,
+    const uint8_t* __restrict__ modality, const uint8_t* __restrict__ time_id, int n_times,
+    int expect_a, int expect_b) {
+  __shared__ float s_lat[EMB_ROWS][EMB_MAXK];
+  __shared__ int s_mod[EMB_ROWS], s_tid[EMB_ROWS];
+  const int rb0 = blockIdx.x * EMB_ROWS;
+  const int nr = min(EMB_ROWS, rows - rb0);
+  if (nr <= 0) return;
+  if (threadIdx.x < nr) {
+    const int r = row0 + rb0 + threadIdx.x;
+    int m = modality[r], t = time_id[r];
+    if ((m != expect_a && m != expect_b) || t >= n_times) {
+      raise_device_error(DEVERR_TAGS);
+      m = expect_a;
+      t = 0;
+    }
+    s_mod[threadIdx.x] = m;
+    s_tid[threadIdx.x] = t;
+  }
+  if (kind == 1) {
+    for (int i = threadIdx.x; i < nr * K; i += blockDim.x)
+      s_lat[i / K][i % K] = lat[(size_t)(rb0 + i / K) * K + (i % K)];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
+    float wr[EMB_MAXK];
+    float bias = 0.f;
+    if (kind == 1) {
+#pragma unroll 8
+      for (int k = 0; k < K; ++k) wr[k] = ld_f32<TW>(w_in + (size_t)c * K + k);
+      bias = ld_f32<TW>(b_in + c);
+    }
+    for (int j = 0; j < nr; ++j) {
+      float acc;
+      if (kind == 1) {
+        acc = bias;
+#pragma unroll 8
+        for (int k = 0; k < K; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
+      } else {
+        acc = text_proj[(size_t)(rb0 + j) * hidden + c];
+      }
+      acc += ld_f32<TW>(mod_emb + (size_t)s_mod[j] * hidden + c) + temb[(size_t)s_tid[j] * hidden + c];
+      x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- timestep MLP
+// Stage 1: h1[t, c] = silu(sum_k feat_t[k] W1[c,k] + b1[c]) with the
+// sinusoidal features of 1000*t computed in shared memory.
+struct Times8 { float t[8]; };
+template <typename TW>
+__global__ void time_mlp1_kernel(Times8 times, int n_times, int t_freq,
+                                 const TW* __restrict__ w1, const TW* __restrict__ b1,
+                                 float* __restrict__ h1, int hidden) {
+  extern __shared__ float s_feat[];  // [n_times][t_freq]
+  const int half = t_freq / 2;
+  for (int i = threadIdx.x; i < n_times * half; i += blockDim.x) {
+    const int t = i / half, j = i % half;
+    const float freq = expf(-logf(10000.0f) * (float)j / (float)half);
+    const float arg = 1000.0f * times.t[t] * freq;
+    float s, c;
+    sincosf(arg, &s, &c);
+    s_feat[t * t_freq + j] = c;
+    s_feat[t * t_freq + half + j] = s;
+  }
+  __syncthreads();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int c = warp; c < hidden; c += nwarps) {
+    for (int t = 0; t < n_times; ++t) {
+      float acc = 0.f;
+      for (int k = lane; k < t_freq; k += 32) acc = fmaf(s_feat[t * t_freq + k], ld_f32<TW>(w1 + (size_t)c * t_freq + k), acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        const float z = acc + ld_f32<TW>(b1 + c);
+        h1[(size_t)t * hidden + c] = z / (1.0f + expf(-z));
+      }
+    }
+  }
+}
+
+// Stage 2: temb[t, c] = sum_k h1[t,k] W2[c,k] + b2[c]; W2 read once.
+constexpr int TMLP_MAXT = 8;
+template <typename TW>
+__global__ void time_mlp2_kernel(const float* __restrict__ h1, int n_times, const TW* __restrict__ w2,
+                                 const TW* __restrict__ b2, float* __restrict__ temb, int hidden) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int c = warp; c < hidden; c += nwarps) {
+    float acc[TMLP_MAXT];
+#pragma unroll
+    for (int t = 0; t < TMLP_MAXT; ++t) acc[t] = 0.f;
+    for (int k = lane; k < hidden; k += 32) {
+      const float wv = ld_f32<TW>(w2 + (size_t)c * hidden + k);
+#pragma unroll
+      for (int t = 0; t < TMLP_MAXT; ++t)
+        if (t < n_times) acc[t] = fmaf(h1[(size_t)t * hidden + k], wv, acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < TMLP_MAXT; ++t) {
+      float a = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0 && t < n_times) temb[(size_t)t * hidden + c] = a + ld_f32<TW>(b2 + c);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- output heads
+// v[r, c] = rstd_r * sum_k x[r,k] g[k] W[c,k] + b[c] for C <= 64 outputs.  A
+// block owns HEAD_ROWS rows; x and g*W are staged in shared memory in chunks
+// of HEAD_KC channels; the row sum of squares is accumulated on the way.
+constexpr int HEAD_ROWS = 64;
+constexpr int HEAD_KC = 64;
+constexpr int HEAD_MAXC = 64;
+template <typename TW>
+__global__ void __launch_bounds__(256) heads_kernel(const float* __restrict__ x, int row0, int rows, int hidden,
+                                                    const TW* __restrict__ g, const TW* __restrict__ w,
+                                                    const TW* __restrict__ b, int C, float eps,
+                                                    float* __restrict__ out) {
+  __shared__ float s_x[HEAD_ROWS][HEAD_KC + 1];
+  __shared__ float s_w[HEAD_MAXC][HEAD_KC + 1];
+  __shared__ float s_ss[HEAD_ROWS];
+  const int rb = blockIdx.x * HEAD_ROWS;
+  const int nr = min(HEAD_ROWS, rows - rb);
+  if (nr <= 0) return;
+  // thread -> (row j, output group): 256 threads = 64 rows x 4 groups of C/4 outputs
+  const int j = threadIdx.x >> 2, grp = threadIdx.x & 3;
+  const int per = (C + 3) / 4;
+  float acc[HEAD_MAXC / 4];
+#pragma unroll
+  for (int i = 0; i < HEAD_MAXC / 4; ++i) acc[i] = 0.f;
+  float ss = 0.f;
+  for (int k0 = 0; k0 < hidden; k0 += HEAD_KC) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < HEAD_ROWS * HEAD_KC; i += blockDim.x) {
+      const int rr = i / HEAD_KC, kk = i % HEAD_KC;
+      s_x[rr][kk] = (rr < nr) ? x[(size_t)(row0 + rb + rr) * hidden + k0 + kk] : 0.f;
+    }
+    for (int i = threadIdx.x; i < C * HEAD_KC; i += blockDim.x) {
+      const int cc = i / HEAD_KC, kk = i % HEAD_KC;
+      s_w[cc][kk] = ld_f32<TW>(w + (size_t)cc * hidden + k0 + kk) * ld_f32<TW>(g + k0 + kk);
+    }
+    __syncthreads();
+    if (grp == 0) {
+      for (int kk = 0; kk < HEAD_KC; ++kk) ss = fmaf(s_x[j][kk], s_x[j][kk], ss);
+    }
+#pragma unroll
+    for (int i = 0; i < HEAD_MAXC / 4; ++i) {
+      const int cc = grp * per + i;
+      if (i < per && cc < C) {
+        float a = acc[i];
+        for (int kk = 0; kk < HEAD_KC; ++kk) a = fmaf(s_x[j][kk], s_w[cc][kk], a);
+        acc[i] = a;
+      }
+    }
+  }
+  if (grp == 0) s_ss[j] = ss;
+  __syncthreads();
+  if (j < nr) {
+    const float rstd = rsqrtf(s_ss[j] / (float)hidden + eps);
+#pragma unroll
+    for (int i = 0; i < HEAD_MAXC / 4; ++i) {
+      const int cc = grp * per + i;
+      if (i < per && cc < C) out[(size_t)(rb + j) * C + cc] = rstd * acc[i] + ld_f32<TW>(b + cc);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- Euler
+struct Clock4 { float dt[4]; };
+__global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v, const uint8_t* __restrict__ mod,
+                             const uint8_t* __restrict__ mask, int n_rows, int width, Clock4 clk) {
+  const size_t total = (size_t)n_rows * width;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / width);
+    if (mask[r]) x[i] = fmaf(clk.dt[mod[r] & 3], v[i], x[i]);
+  }
+}
+
+// ================================================================ host launchers
+
+static int grid_for_rows(int rows, int per_sm) {
+  const int g = num_sms() * per_sm;
+  return rows < g ? (rows > 0 ? rows : 1) : g;
+}
+
+fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st) {
+  const int total = T * H * W;
+  const int blocks = (total + 255) / 256;
+  keep_map_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(T, H, W, keep_idx, near_idx);
+  return cuda_check(cudaGetLastError(), "keep_map_kernel");
+}
+
+fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
+                           int n_keep, int n_grid, int n_rows, int hidden, cudaStream_t st) {
+  const int n_out = n_keep + (n_rows - n_grid);
+  gather_rows_kernel<<<grid_for_rows(n_out, 8), 256, 0, st>>>(x, pos, xc, posc, keep_idx, n_keep, n_grid, n_out,
+                                                              hidden);
+  return cuda_check(cudaGetLastError(), "gather_rows_kernel");
+}
+
+fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
+                              const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
+                              cudaStream_t st) {
+  const int g = grid_for_rows(n_rows, 8);
+  if (out != x) {
+    broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 0);
+    return cuda_check(cudaGetLastError(), "broadcast_kernel");
+  }
+  broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 1);
+  fsdit_status s = cuda_check(cudaGetLastError(), "broadcast_kernel(dropped rows)");
+  if (s != FSDIT_OK) return s;
+  broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 2);
+  return cuda_check(cudaGetLastError(), "broadcast_kernel(kept rows)");
+}
+
+fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
+                                 cudaStream_t st) {
+  const int grid = grid_for_rows(rows, 8);
+  if (dtype == FSDIT_BF16)
+    rmsnorm_cast_kernel<bf16><<<grid, 256, 0, st>>>(x, (const bf16*)g, (bf16*)xn, rows, hidden, eps);
+  else
+    rmsnorm_cast_kernel<float><<<grid, 256, 0, st>>>(x, (const float*)g, (float*)xn, rows, hidden, eps);
+  return cuda_check(cudaGetLastError(), "rmsnorm_cast_kernel");
+}
+
+template <typename TW>
+static fsdit_status embed_t(float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
+                            const void* w_in, const void* b_in, const float* text_proj, const void* mod_emb,
+                            const float* temb, const uint8_t* modality, const uint8_t* time_id, int n_times,
+                            int ea, int eb, cudaStream_t st) {
+  if (rows <= 0) return FSDIT_OK;
+  const int blocks = (rows + EMB_ROWS - 1) / EMB_ROWS;
+  embed_kernel<TW><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in, (const TW*)b_in,
+                                           text_proj, (const TW*)mod_emb, temb, modality, time_id, n_times, ea, eb);
+  return cuda_check(cudaGetLastError(), "embed_kernel");
+}
+
+fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
+                          const void* w_in, const void* b_in, const float* text_proj, const void* mod_emb,
+                          const float* temb, const uint8_t* modality, const uint8_t* time_id, int n_times, int ea,
+                          int eb, cudaStream_t st) {
+  if (dtype == FSDIT_BF16)
+    return embed_t<bf16>(x, hidden, row0, rows, kind, lat, K, w_in, b_in, text_proj, mod_emb, temb, modality,
+                         time_id, n_times, ea, eb, st);
+  return embed_t<float>(x, hidden, row0, rows, kind, lat, K, w_in, b_in, text_proj, mod_emb, temb, modality,
+                        time_id, n_times, ea, eb, st);
+}
+
+fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, int t_freq, const void* w1,
+                             const void* b1, const void* w2, const void* b2, float* h1, float* temb, int hidden,
+                             cudaStream_t st) {
+  const int blocks = num_sms() * 2;
+  const size_t sm1 = (size_t)n_times * t_freq * sizeof(float);
+  Times8 times_dev;
+  for (int i = 0; i < 8; ++i) times_dev.t[i] = i < n_times ? times_host[i] : 0.f;
+  if (dtype == FSDIT_BF16) {
+    time_mlp1_kernel<bf16><<<blocks, 256, sm1, st>>>(times_dev, n_times, t_freq, (const bf16*)w1, (const bf16*)b1,
+                                                     h1, hidden);
+    time_mlp2_kernel<bf16><<<blocks, 256, 0, st>>>(h1, n_times, (const bf16*)w2, (const bf16*)b2, temb, hidden);
+  } else {
+    time_mlp1_kernel<float><<<blocks, 256, sm1, st>>>(times_dev, n_times, t_freq, (const float*)w1,
+                                                      (const float*)b1, h1, hidden);
+    time_mlp2_kernel<float><<<blocks, 256, 0, st>>>(h1, n_times, (const float*)w2, (const float*)b2, temb, hidden);
+  }
+  return cuda_check(cudaGetLastError(), "time_mlp kernels");
+}
+
+fsdit_status launch_heads(int dtype, const float* x, int row0, int rows, int hidden, const void* g, const void* w,
+                          const void* b, int C, float eps, float* out, cudaStream_t st) {
+  if (rows <= 0) return FSDIT_OK;
+  const int blocks = (rows + HEAD_ROWS - 1) / HEAD_ROWS;
+  if (dtype == FSDIT_BF16)
+    heads_kernel<bf16><<<blocks, 256, 0, st>>>(x, row0, rows, hidden, (const bf16*)g, (const bf16*)w,
+                                               (const bf16*)b, C, eps, out);
+  else
+    heads_kernel<float><<<blocks, 256, 0, st>>>(x, row0, rows, hidden, (const float*)g, (const float*)w,
+                                                (const float*)b, C, eps, out);
+  return cuda_check(cudaGetLastError(), "heads_kernel");
+}
+
+fsdit_status launch_euler(float* x, const float* v, const uint8_t* mod, const uint8_t* mask, int n_rows, int width,
+                          const float* t_cur, const float* t_next, cudaStream_t st) {
+  Clock4 c;
+  for (int i = 0; i < 4; ++i) c.dt[i] = t_next[i] - t_cur[i];
+  const size_t total = (size_t)n_rows * width;
+  size_t blocks = (total + 255) / 256;
+  const size_t cap = (size_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks == 0) blocks = 1;
+  euler_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, v, mod, mask, n_rows, width, c);
+  return cuda_check(cudaGetLastError(), "euler_kernel");
+}
+
+}  // namespace fsdit

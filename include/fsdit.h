@@ -1,0 +1,275 @@
+/*
+ * fsdit.h -- C ABI of libfsdit.so: the few-step Flash DiT hot path on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources: web write-ups of arXiv 2609.15863 ("LynnReal-Omni"):
+ *   [tokendh]    tokendh.com news article, sections "一个模型如何同时干七件事：
+ *                原生多模态骨干网络" (backbone, per-row tags) and "训练的核心
+ *                难题：怎么让模型又快又准" (flow matching, dual clocks, Flash
+ *                layer schedule, spatial token compression);
+ *   [PaperDaily] longzhangge PaperDaily "LynnReal Lab视频恢复与生成：统一多模态
+ *                控制，Flash降至377毫秒", section 一 (tags, control offset,
+ *                separate clocks) and section 二 "Flash怎么把22帧压到377毫秒"
+ *                (compression, nearest-kept update broadcast, fused ops).
+ *
+ * Conventions for every call
+ *  - Memory: the caller owns every buffer.  Pointers marked (device) are CUDA
+ *    device pointers, 16-byte aligned; (host) are host pointers.  The library
+ *    allocates nothing on these paths; scratch comes from a caller-provided
+ *    workspace whose size fsdit_*_workspace_size() returns.
+ *  - Streams: calls enqueue kernels on `stream` and return without waiting.
+ *    All argument checks run on the host before any launch; a failed check
+ *    launches nothing.
+ *  - Errors: every call returns an fsdit_status; fsdit_last_error() gives a
+ *    thread-local message for the last failure.  Kernels never trap: a device
+ *    wait that exceeds its bound sets a device error word that
+ *    fsdit_device_error() reads (after synchronizing the stream).
+ *  - Layout: activations are token-major, row-major [rows, hidden].  Linear
+ *    weights are [out_features, in_features] row-major (K contiguous), so a
+ *    projection is y = x W^T + b.  The residual stream is float32 in every
+ *    configuration; `dtype` selects the type of weights, biases, norm gains,
+ *    text features and GEMM operands (FSDIT_F32 or FSDIT_BF16).
+ *  - Packed sequence: rows [0, n_vrows) are video latent rows (the target grid
+ *    first, then clean control frames), then n_text text rows, then n_audio
+ *    audio rows.  Per-row tags ([tokendh] backbone section; [PaperDaily] 一):
+ *    modality (0 text, 1 video, 2 audio, 3 video control), a noise-time slot
+ *    into a per-call time table, a 3D (t,h,w) RoPE position and an output
+ *    mark.
+ */
+#ifndef FSDIT_H
+#define FSDIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FSDIT_API __attribute__((visibility("default")))
+#else
+#define FSDIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fsdit_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  FSDIT_OK = 0,
+  FSDIT_E_NULL = -1,      /* a required pointer is NULL */
+  FSDIT_E_SHAPE = -2,     /* sizes inconsistent or outside what the kernels handle */
+  FSDIT_E_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+  FSDIT_E_DTYPE = -4,     /* unknown dtype */
+  FSDIT_E_CUDA = -5,      /* a CUDA runtime/driver call failed (message says which) */
+  FSDIT_E_WORKSPACE = -6, /* workspace smaller than fsdit_*_workspace_size() */
+  FSDIT_E_TIMEOUT = -7    /* a kernel gave up a bounded device wait */
+} fsdit_status;
+
+typedef enum { FSDIT_F32 = 0, FSDIT_BF16 = 1 } fsdit_dtype;
+
+enum { FSDIT_MOD_TEXT = 0, FSDIT_MOD_VIDEO = 1, FSDIT_MOD_AUDIO = 2, FSDIT_MOD_CONTROL = 3 };
+
+/* Model dimensions.  [tokendh] backbone section: hidden 5376, 56 heads of
+ * 128, FFN 14336 (the Flash model keeps 42 of the 50 layers).  The head
+ * dimension must be 128; rope_split gives the (t,h,w) chunk widths of a head
+ * (32/48/48), each even, summing to head_dim.  hidden must be a multiple of 64
+ * and equal heads*head_dim; ffn a multiple of 64. */
+typedef struct {
+  int hidden, heads, head_dim, ffn;
+  int rope_split[3];
+  float rms_eps;    /* RMSNorm epsilon (1e-6) */
+  float rope_theta; /* RoPE base (10000) */
+  int dtype;        /* fsdit_dtype of weights and GEMM operands */
+} fsdit_dims;
+
+/* Weights of one pre-norm DiT block (all (device), `dtype`).
+ *   w_qkv [3*hidden, hidden]  rows: q (hidden), k (hidden), v (hidden); head h
+ *                             owns rows [h*128, h*128+128) of each part
+ *   b_qkv [3*hidden]
+ *   w_o   [hidden, hidden],  b_o [hidden]
+ *   w_1   [ffn, hidden],     b_1 [ffn]
+ *   w_2   [hidden, ffn],     b_2 [hidden]
+ *   g_attn, g_ffn [hidden]   RMSNorm gains */
+typedef struct {
+  const void *w_qkv, *b_qkv, *w_o, *b_o, *w_1, *b_1, *w_2, *b_2, *g_attn, *g_ffn;
+} fsdit_block_weights;
+
+/* Embedding, timestep-MLP and output-head weights (all (device), `dtype`).
+ *   w_vin [hidden, c_video], b_vin   video/control latent -> hidden
+ *   w_tin [hidden, c_text],  b_tin   text feature -> hidden
+ *   w_ain [hidden, c_audio], b_ain   audio latent -> hidden
+ *   mod_emb [4, hidden]              learned modality embedding
+ *   w_t1 [hidden, t_freq], b_t1, w_t2 [hidden, hidden], b_t2   timestep MLP
+ *   g_out [hidden]                   final RMSNorm gain
+ *   w_vout [c_video, hidden], b_vout; w_aout [c_audio, hidden], b_aout */
+typedef struct {
+  const void *w_vin, *b_vin, *w_tin, *b_tin, *w_ain, *b_ain, *mod_emb;
+  const void *w_t1, *b_t1, *w_t2, *b_t2;
+  const void *g_out, *w_vout, *b_vout, *w_aout, *b_aout;
+  int c_video, c_text, c_audio, t_freq;
+} fsdit_io_weights;
+
+/* Tags of a packed sequence (all arrays (device)).
+ *   n_tokens = n_vrows + n_text + n_audio
+ *   grid_t/h/w: the target video grid, rows [0, grid_t*grid_h*grid_w) in
+ *     (t,h,w) row-major order (0,0,0 if there is none); control rows follow.
+ *   keep_idx [n_keep], near_idx [grid rows]: keep-index map of that grid from
+ *     fsdit_build_keep_map (NULL/0: no compression).
+ *   pos_thw [n_tokens][3] int32, modality/time_id/out_mask [n_tokens] uint8. */
+typedef struct {
+  int n_tokens, n_vrows, n_text, n_audio;
+  int grid_t, grid_h, grid_w;
+  const int32_t* pos_thw;
+  const uint8_t* modality;
+  const uint8_t* time_id;
+  const uint8_t* out_mask;
+  const int32_t* keep_idx;
+  int n_keep;
+  const int32_t* near_idx;
+} fsdit_tokens;
+
+/* ---------------------------------------------------------------- queries */
+
+FSDIT_API const char* fsdit_last_error(void);
+FSDIT_API const char* fsdit_version(void);
+
+/* Synchronizes `stream`, returns FSDIT_E_TIMEOUT if any kernel since the last
+ * reset gave up a bounded wait (and clears the word), else FSDIT_OK. */
+FSDIT_API fsdit_status fsdit_device_error(fsdit_stream_t stream);
+
+/* Number of kept tokens of a T x H x W grid: T * (H/2+1) * (W/2+1). */
+FSDIT_API int fsdit_keep_count(int T, int H, int W);
+
+/* Workspace bytes for dit_block_forward on n_tokens rows (n_keep kept grid
+ * rows, 0 = no compression) and for one dit_stack_forward / dit_flow_sample
+ * call. */
+FSDIT_API size_t fsdit_block_workspace_size(const fsdit_dims* dims, int n_tokens, int n_keep);
+FSDIT_API size_t fsdit_stack_workspace_size(const fsdit_dims* dims, const fsdit_io_weights* io,
+                                  const fsdit_tokens* tok, int n_times);
+
+/* ---------------------------------------------------------------- hot path */
+
+/* Keep-index map of a T x H x W video grid ([tokendh] training section,
+ * Flash paragraph; [PaperDaily] 二): per frame keep rows {0,2,4,..}+{H-1} and
+ * columns {0,2,4,..}+{W-1}, no temporal drop.  keep_idx[c] (device, int32
+ * [fsdit_keep_count]) = full-grid row id t*H*W+h*W+w of kept token c in
+ * (t, kept h, kept w) order; near_idx[p] (device, int32 [T*H*W]) = compact id
+ * of the kept token nearest to row p in its own frame (a dropped index lies
+ * midway between two kept ones; the lower one is taken). */
+FSDIT_API fsdit_status fsdit_build_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx,
+                                  fsdit_stream_t stream);
+
+/* Gather the compressed sequence: rows [0, n_keep) of x_c / pos_c are the
+ * grid rows keep_idx[c] of x / pos; rows [n_keep, n_keep + n_rows - n_grid)
+ * are the non-grid rows n_grid.. n_rows-1 in order (text and audio are never
+ * compressed, [PaperDaily] 二).  x, x_c float32 [.., hidden] (device); pos,
+ * pos_c int32 [..,3] (device, may both be NULL). */
+FSDIT_API fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, float* x_c, int32_t* pos_c,
+                               const int32_t* keep_idx, int n_keep, int n_grid, int n_rows,
+                               int hidden, fsdit_stream_t stream);
+
+/* Nearest-kept broadcast + residual ([PaperDaily] 二; [tokendh] training
+ * section): the compressed layers' update of kept token c is
+ * d_c = y_c[c] - x[keep_idx[c]]; kept grid rows take y_c, dropped grid rows p
+ * take x[p] + d_{near_idx[p]} (float32 arithmetic), non-grid rows take their
+ * y_c rows.  out may equal x (then it runs in two ordered launches). */
+FSDIT_API fsdit_status fsdit_broadcast_residual(const float* x, const float* y_c, float* out,
+                                      const int32_t* keep_idx, const int32_t* near_idx,
+                                      int n_keep, int n_grid, int n_rows, int hidden,
+                                      fsdit_stream_t stream);
+
+/* RMSNorm fused into the GEMM-operand pass: xn[r] = cast(x[r] * g /
+ * sqrt(mean(x[r]^2) + eps)).  x float32 [rows, hidden]; g and xn in `dtype`. */
+FSDIT_API fsdit_status fsdit_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden,
+                                float eps, int dtype, fsdit_stream_t stream);
+
+/* Epilogues of fsdit_linear (all add the bias first):
+ *   FSDIT_EPI_BIAS       out (dtype)  = acc + b
+ *   FSDIT_EPI_BIAS_F32   out (f32)    = acc + b
+ *   FSDIT_EPI_QKV_ROPE   out (dtype)  = rope(acc + b) on columns < 2*hidden
+ *                        (q and k), per row position pos[row]
+ *   FSDIT_EPI_GELU       out (dtype)  = gelu_tanh(acc + b)
+ *   FSDIT_EPI_RESIDUAL   out (f32)    = resid + acc + b   (out may equal resid) */
+enum {
+  FSDIT_EPI_BIAS = 0,
+  FSDIT_EPI_BIAS_F32 = 1,
+  FSDIT_EPI_QKV_ROPE = 2,
+  FSDIT_EPI_GELU = 3,
+  FSDIT_EPI_RESIDUAL = 4
+};
+
+/* One projection out[M,N] = a[M,K] w[N,K]^T with a fused epilogue.
+ * a, w, b in `dtype` (device).  bf16 runs on the tcgen05 tensor cores (TMA
+ * operand staging, fp32 accumulation in tensor memory); f32 runs exact fp32
+ * FMA.  K % 8 == 0; N % 32 == 0.  dims supplies head_dim / rope split / theta
+ * for FSDIT_EPI_QKV_ROPE (pos int32 [M][3] (device)). */
+FSDIT_API fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, const void* b,
+                          void* out, const float* resid, const int32_t* pos, int M, int N, int K,
+                          int epilogue, fsdit_stream_t stream);
+
+/* Joint attention ([tokendh] backbone section: one sequence of text,
+ * video and audio tokens through one denoiser): for each head,
+ * softmax(q k^T / sqrt(128)) v over all n rows, no mask.  qkv [n, 3*hidden]
+ * in `dtype` (q | k | v, RoPE already applied); out [n, hidden] in `dtype`. */
+FSDIT_API fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n,
+                             fsdit_stream_t stream);
+
+/* One DiT block.  x_in, x_out float32 [n_tokens, hidden] (device);
+ * x_out may equal x_in.  With tok->keep_idx != NULL the block is the Flash
+ * compressed block in per-block form: gather the kept grid rows and all
+ * non-grid rows, run the block on them, broadcast with
+ * fsdit_broadcast_residual.  Positions of kept rows stay their original
+ * (t,h,w). */
+FSDIT_API fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_block_weights* w,
+                               const fsdit_tokens* tok, const float* x_in, float* x_out,
+                               void* workspace, size_t ws_bytes, fsdit_stream_t stream);
+
+/* One backbone evaluation: embedding (input projections + modality
+ * embedding + timestep embedding of time_table[time_id[row]]), n_layers
+ * blocks (layers: host array of n_layers weight structs; layer_compress: host
+ * uint8 [n_layers], 1 = token-compressed; a run of compressed layers gathers
+ * once and broadcasts once, which equals the per-layer form in exact
+ * arithmetic), final RMSNorm and the video/audio velocity heads.
+ *   time_table (host) float [n_times], n_times <= 8
+ *   video_lat float32 [n_vrows, c_video], audio_lat float32 [n_audio, c_audio],
+ *   text_emb `dtype` [n_text, c_text]                      (device, inputs)
+ *   v_video float32 [n_vrows, c_video], v_audio float32 [n_audio, c_audio]
+ *                                                           (device, outputs) */
+FSDIT_API fsdit_status dit_stack_forward(const fsdit_dims* dims, int n_layers,
+                               const fsdit_block_weights* layers, const uint8_t* layer_compress,
+                               const fsdit_io_weights* io, const fsdit_tokens* tok,
+                               const float* time_table, int n_times, const float* video_lat,
+                               const void* text_emb, const float* audio_lat, float* v_video,
+                               float* v_audio, void* workspace, size_t ws_bytes,
+                               fsdit_stream_t stream);
+
+/* One flow-matching Euler step with a clock per modality ([tokendh]
+ * training section: x_t = (1-t) x0 + t eps, the network predicts
+ * v = eps - x0; [PaperDaily] 一: video and audio share the forward but keep
+ * their own noise clocks): for each row r with out_mask[r] != 0,
+ * x[r] += (t_next[m] - t_cur[m]) * v[r], m = row_modality[r].  x, v float32
+ * [n_rows, row_width] (device); row_modality, out_mask uint8 [n_rows]
+ * (device); t_cur, t_next (host) float [4] indexed by modality code. */
+FSDIT_API fsdit_status flow_euler_step(float* x, const float* v, const uint8_t* row_modality,
+                             const uint8_t* out_mask, int n_rows, int row_width,
+                             const float* t_cur, const float* t_next, fsdit_stream_t stream);
+
+/* The few-step sampler: n_evals evaluations of dit_stack_forward; eval e
+ * uses time table {0, t_video[e], t_audio[e]} (slots 0 clean, 1 video, 2 audio)
+ * and then Euler-steps the video rows from t_video[e] to t_video[e+1] and the
+ * audio rows from t_audio[e] to t_audio[e+1].  Flash: 3 evaluations on
+ * 0.2 -> 0.0769 -> 0.027 -> 0 (video) and 0.5 -> 0.25 -> 0.1 -> 0 (audio)
+ * ([tokendh] training section).  video_lat / audio_lat (device, float32) are
+ * updated in place; t_video, t_audio (host) float [n_evals + 1]. */
+FSDIT_API fsdit_status dit_flow_sample(const fsdit_dims* dims, int n_layers,
+                             const fsdit_block_weights* layers, const uint8_t* layer_compress,
+                             const fsdit_io_weights* io, const fsdit_tokens* tok, int n_evals,
+                             const float* t_video, const float* t_audio, float* video_lat,
+                             const void* text_emb, float* audio_lat, void* workspace,
+                             size_t ws_bytes, fsdit_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FSDIT_H */

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/fsdit.h declares, and rejects bad arguments on the
+host before any launch (no compute call is made here)."""
+
+import ctypes as C
+
+import pytest
+
+from few_step_dit_b200 import api, build, lib as L
+
+
+@pytest.fixture(scope="module")
+def fs():
+    build.build()
+    return L.load()
+
+
+def test_library_exports_every_declared_symbol(fs):
+    names = L.header_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(fs, n), n
+    assert set(names) == set(L._SIGS), "binding signatures out of sync with the header"
+
+
+def test_keep_count_closed_form(fs):
+    assert fs.fsdit_keep_count(6, 34, 60) == 3348
+    assert fs.fsdit_keep_count(2, 9, 10) == 60
+    assert fs.fsdit_keep_count(1, 1, 1) == 1
+    assert fs.fsdit_keep_count(0, 9, 10) == 0
+
+
+def _dims(**kw):
+    d = api.make_dims(5376, 42, 14336, L.BF16)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_size_rejects_bad_dims(fs):
+    assert fs.fsdit_block_workspace_size(C.byref(_dims()), 12560, 3348) > 0
+    assert fs.fsdit_block_workspace_size(C.byref(_dims(head_dim=64)), 100, 0) == 0
+    assert fs.fsdit_block_workspace_size(C.byref(_dims(dtype=7)), 100, 0) == 0
+    assert fs.fsdit_block_workspace_size(C.byref(_dims(ffn=100)), 100, 0) == 0
+
+
+def test_block_workspace_grows_with_rows(fs):
+    d = _dims()
+    a = fs.fsdit_block_workspace_size(C.byref(d), 3668, 0)
+    b = fs.fsdit_block_workspace_size(C.byref(d), 12560, 0)
+    assert b > a > 0
+    # bf16 GEMM operands + fp32 compressed residual
+    H, F = 5376, 14336
+    assert b >= 12560 * (H + 3 * H + F) * 2
+
+
+def test_entry_points_reject_null_and_bad_shapes_without_launching(fs):
+    d = _dims()
+    s = None
+    assert fs.fsdit_linear(C.byref(d), None, None, None, None, None, None, 8, 64, 64, 0, s) == -1
+    fake = C.c_void_p(0x10000)            # never dereferenced: validation fails first
+    odd = C.c_void_p(0x10004)
+    assert fs.fsdit_linear(C.byref(d), odd, fake, fake, fake, None, None, 8, 64, 64, 0, s) == -3
+    assert fs.fsdit_linear(C.byref(d), fake, fake, fake, fake, None, None, 8, 60, 64, 0, s) == -2
+    assert fs.fsdit_linear(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 60, 0, s) == -2
+    assert fs.fsdit_linear(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 64, 9, s) == -2
+    # RoPE epilogue needs N == 3*hidden and a position array
+    assert fs.fsdit_linear(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 64, 2, s) == -1
+    assert fs.fsdit_build_keep_map(0, 9, 10, fake, fake, s) == -2
+    assert fs.fsdit_gather_rows(fake, None, fake, None, fake, 0, 10, 10, 64, s) == -2
+    assert fs.fsdit_broadcast_residual(fake, fake, fake, fake, fake, 5, 4, 10, 64, s) == -2
+    assert fs.fsdit_rmsnorm_cast(fake, fake, fake, 4, 100, 1e-6, 1, s) == -2
+    assert fs.fsdit_rmsnorm_cast(fake, fake, fake, 4, 64, 1e-6, 3, s) == -4
+    tc = (C.c_float * 4)(0, 0.2, 0.5, 0)
+    assert fs.flow_euler_step(fake, fake, None, None, 4, 24, tc, tc, s) == -1
+    assert fs.flow_euler_step(fake, fake, fake, fake, 4, 0, tc, tc, s) == -2
+    msg = L.last_error()
+    assert "row_width" in msg
+
+
+def test_block_forward_rejects_inconsistent_tokens(fs):
+    d = _dims()
+    fake = C.c_void_p(0x10000)
+    w = L.BlockWeights(*([0x10000] * 10))
+    tok = L.Tokens()
+    tok.n_tokens, tok.n_vrows, tok.n_text, tok.n_audio = 100, 80, 10, 5   # 95 != 100
+    tok.pos_thw = 0x10000
+    assert fs.dit_block_forward(C.byref(d), C.byref(w), C.byref(tok), fake, fake, fake, 1 << 30, None) == -2
+    tok.n_audio = 10
+    tok.grid_t, tok.grid_h, tok.grid_w = 1, 9, 10                           # 90 > 80 video rows
+    assert fs.dit_block_forward(C.byref(d), C.byref(w), C.byref(tok), fake, fake, fake, 1 << 30, None) == -2
+    tok.grid_t, tok.grid_h, tok.grid_w = 1, 8, 10
+    tok.keep_idx, tok.near_idx, tok.n_keep = 0x10000, 0x10000, 7            # should be 30
+    assert fs.dit_block_forward(C.byref(d), C.byref(w), C.byref(tok), fake, fake, fake, 1 << 30, None) == -2
+    tok.n_keep = 30
+    # workspace too small
+    assert fs.dit_block_forward(C.byref(d), C.byref(w), C.byref(tok), fake, fake, fake, 16, None) == -6

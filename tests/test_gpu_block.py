@@ -1,0 +1,171 @@
+"""Block, stack and sampler parity of the CUDA path against the oracle.
+
+fp32 workloads: relative L2 <= 1e-5.  bf16 workloads (bf16 weights and GEMM
+operands, fp32 accumulation and residual stream): relative L2 <= 1e-2 per
+block and per full denoise.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from few_step_dit_b200 import api, build, lib as L
+from few_step_dit_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    L.load()
+    yield
+    torch.cuda.synchronize()
+    api.device_error()
+
+
+def _np(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _setup(w, n_layers=None):
+    layers, io = S.make_weights(w, n_layers=n_layers)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    return layers, io, inp, tags
+
+
+def _oracle_tok(w, tags):
+    tok = dict(tags)
+    if any(w.compress):
+        k, n = O.keep_map(*w.grid)
+        tok["keep_idx"], tok["near_idx"] = k, n
+    return tok
+
+
+def _block_case(w, compress):
+    layers, io, inp, tags = _setup(w, n_layers=1)
+    seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
+    bw = api.BlockWeights({k: v.to(DEV) for k, v in layers[0].items()})
+    dims = api.dims_of(w)
+    x = inp["x"].float()
+    out = api.block_forward(dims, bw, seq, x.to(DEV), compress=compress)
+    torch.cuda.synchronize()
+    wn = S.to_numpy64(layers[0])
+    xn = x.double().numpy()
+    if compress:
+        k, n = O.keep_map(*w.grid)
+        ref = O.dit_block_compressed(xn, wn, tags["pos"], w.heads, w.head_dim, k, n, w.n_video)
+    else:
+        ref = O.dit_block(xn, wn, tags["pos"], w.heads, w.head_dim)
+    return _np(out), ref, xn
+
+
+@pytest.mark.parametrize("compress", [True, False])
+def test_tiny_fp32_block(compress):
+    w = S.WORKLOADS["tiny_block_f32"]
+    got, ref, x = _block_case(w, compress)
+    err = O.rel_l2(got, ref)
+    assert err < 1e-5, err
+    # the block's update itself (y - x) meets the bound too
+    assert O.rel_l2(got - x, ref - x) < 1e-5
+
+
+def test_tiny_fp32_block_in_place_compressed():
+    w = S.WORKLOADS["tiny_block_f32"]
+    layers, io, inp, tags = _setup(w, n_layers=1)
+    seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
+    bw = api.BlockWeights({k: v.to(DEV) for k, v in layers[0].items()})
+    x = inp["x"].float().to(DEV)
+    ref = api.block_forward(api.dims_of(w), bw, seq, x.clone())
+    api.block_forward(api.dims_of(w), bw, seq, x, x_out=x)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, x)
+
+
+@pytest.mark.parametrize("grid", [(2, 9, 10), (3, 6, 7)])
+@pytest.mark.parametrize("compress", [True, False])
+def test_bf16_block_small_width(grid, compress):
+    w = S.scaled(S.WORKLOADS["flash_block_6x34x60"], hidden=256, heads=2, ffn=512, grid=grid,
+                 n_text=16, n_audio=8)
+    got, ref, x = _block_case(w, compress)
+    err = O.rel_l2(got, ref)
+    assert err < 1e-2, err
+    assert O.rel_l2(got - x, ref - x) < 1e-2
+
+
+def test_tiny_fp32_euler_step_from_block_velocity():
+    # one Euler step video 0.2 -> 0.0769, audio 0.5 -> 0.25 on the tiny workload
+    w = S.WORKLOADS["tiny_block_f32"]
+    g = torch.Generator().manual_seed(7)
+    n_vrows = w.n_video
+    x = torch.randn(n_vrows, w.video_ch, generator=g)
+    v = torch.randn(n_vrows, w.video_ch, generator=g)
+    tags = S.pack_tokens(w)
+    mod = torch.as_tensor(tags["video_modality"])
+    mask = torch.as_tensor(tags["video_out"])
+    tc, tn = [0, 0.2, 0.5, 0], [0, 0.0769, 0.25, 0]
+    xd = x.to(DEV)
+    api.euler_step(xd, v.to(DEV), mod.to(DEV), mask.to(DEV), tc, tn)
+    torch.cuda.synchronize()
+    ref = O.euler_step(x.numpy(), v.numpy(), mod.numpy(), mask.numpy(), tc, tn)
+    assert O.rel_l2(_np(xd), ref) < 1e-6
+
+
+def _stack_case(w, n_layers, time_table):
+    layers, io, inp, tags = _setup(w)
+    dims = api.dims_of(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(dims, [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vv, va = bb.forward(seq, time_table, inp["video_lat"].to(DEV), inp["text_emb"].to(DEV),
+                        inp["audio_lat"].to(DEV))
+    torch.cuda.synchronize()
+    tok = _oracle_tok(w, tags)
+    ln = [S.to_numpy64(l) for l in layers]
+    ion = S.to_numpy64(io)
+    rv, ra = O.dit_stack(ln, w.compress, ion, tok, time_table, _np(inp["video_lat"]),
+                         _np(inp["text_emb"]), _np(inp["audio_lat"]), w.heads, w.head_dim)
+    return (_np(vv), _np(va)), (rv, ra)
+
+
+def test_tiny_fp32_stack_with_compressed_segment():
+    w = S.scaled(S.WORKLOADS["tiny_block_f32"], n_layers=6, compress=(0, 1, 1, 1, 0, 0))
+    (gv, ga), (rv, ra) = _stack_case(w, 6, [0.0, 0.2, 0.5])
+    assert O.rel_l2(gv, rv) < 1e-5
+    assert O.rel_l2(ga, ra) < 1e-5
+
+
+def test_bf16_stack_small_width():
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=8,
+                 compress=(0, 0, 1, 1, 1, 1, 0, 0))
+    (gv, ga), (rv, ra) = _stack_case(w, 8, [0.0, 0.2, 0.5])
+    assert O.rel_l2(gv, rv) < 1e-2
+    assert O.rel_l2(ga, ra) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sampler_matches_oracle(dtype):
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=6,
+                 compress=(0, 1, 1, 1, 0, 0), dtype=dtype)
+    layers, io, inp, tags = _setup(w)
+    dims = api.dims_of(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(dims, [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vl, al = inp["video_lat"].to(DEV).clone(), inp["audio_lat"].to(DEV).clone()
+    bb.sample(seq, w.video_clock, w.audio_clock, vl, inp["text_emb"].to(DEV), al)
+    torch.cuda.synchronize()
+    tok = _oracle_tok(w, tags)
+    rv, ra = O.flow_sample([S.to_numpy64(l) for l in layers], w.compress, S.to_numpy64(io), tok,
+                           w.video_clock, w.audio_clock, _np(inp["video_lat"]), _np(inp["text_emb"]),
+                           _np(inp["audio_lat"]), w.heads, w.head_dim)
+    bound = 1e-5 if dtype == "f32" else 1e-2
+    # the latents move by sum(dt * v); compare the total update too
+    assert O.rel_l2(_np(vl), rv) < bound
+    assert O.rel_l2(_np(al), ra) < bound
+    assert O.rel_l2(_np(vl) - _np(inp["video_lat"]), rv - _np(inp["video_lat"])) < bound
