@@ -46,7 +46,7 @@ def flash_layer_compress(n_full_head=2, n_comp=26, n_full_tail=14):
 
 
 # ---------------------------------------------------------------------------
-# a1. Keep-index map  [tokendh, training section, Flash paragraph: 2x spatial
+# Keep-index map  [tokendh, training section, Flash paragraph: 2x spatial
 # down-sampling that keeps the border rows/columns; PaperDaily section 二:
 # every other video token along each spatial axis of every frame, edge rows
 # and columns kept, no temporal drop].
@@ -181,7 +181,7 @@ def linear(x, w, b=None):
 
 
 # ---------------------------------------------------------------------------
-# a4-a8. One DiT block (uncompressed).
+# One DiT block (uncompressed).
 # ---------------------------------------------------------------------------
 
 def dit_block(x, w, pos, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
@@ -210,7 +210,7 @@ def dit_block(x, w, pos, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
 
 
 # ---------------------------------------------------------------------------
-# a3, a9. Compressed block: gather kept rows, run the block, broadcast back.
+# Compressed block: gather kept rows, run the block, broadcast back.
 # ---------------------------------------------------------------------------
 
 def gather_rows(x, keep_idx, n_video):
@@ -263,7 +263,7 @@ def dit_block_compressed(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video
 
 
 # ---------------------------------------------------------------------------
-# a2. Embedding, a11 heads.
+# Embedding and output heads.
 # ---------------------------------------------------------------------------
 
 def timestep_features(t, dim=256, max_period=10000.0):
@@ -327,7 +327,7 @@ def output_heads(x, io, modality, eps=1e-6):
 
 
 # ---------------------------------------------------------------------------
-# a10. Backbone stack.
+# Backbone stack.
 # ---------------------------------------------------------------------------
 
 def dit_stack(layers, layer_compress, io, tok, time_table, video_lat, text_emb,
@@ -372,7 +372,7 @@ def dit_stack(layers, layer_compress, io, tok, time_table, video_lat, text_emb,
 
 
 # ---------------------------------------------------------------------------
-# a12, a13. Flow matching and the Euler loop.
+# Flow matching and the Euler loop.
 # ---------------------------------------------------------------------------
 
 def flow_interpolate(x0, eps_noise, t):
