@@ -162,7 +162,7 @@ def linear(dims, a, w, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, s
 def attention(dims, qkv, out=None, stream=None):
     n = qkv.shape[0]
     if out is None:
-        out = torch.empty(n, dims.hidden, dtype=qkv.dtype, device=qkv.device)
+        out = torch.empty(n, dims.heads * dims.head_dim, dtype=qkv.dtype, device=qkv.device)
     L.call("fsdit_attention", C.byref(dims), L.ptr(qkv), L.ptr(out), n, _stream(stream))
     return out
 

@@ -5,10 +5,38 @@
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
 namespace fsdit {
+
+// ---------------------------------------------------------------- profiler
+static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "gemm_gelu", "gemm_bias_f32",
+                                           "gemm_bias",     "attention",     "rmsnorm_cast", "gather",
+                                           "broadcast",     "embed",         "time_mlp",  "heads",
+                                           "euler",         "keep_map"};
+struct Prof {
+  bool on = false;
+  int used = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> cls, kernels;
+  std::vector<double> flops, bytes;
+};
+static Prof g_prof;
+
+ProfScope::ProfScope(int c, int k, double fl, double by, cudaStream_t s) : slot(-1), st(s) {
+  if (!g_prof.on || 2 * (size_t)(g_prof.used + 1) > g_prof.ev.size()) return;
+  slot = g_prof.used++;
+  g_prof.cls[slot] = c;
+  g_prof.kernels[slot] = k;
+  g_prof.flops[slot] = fl;
+  g_prof.bytes[slot] = by;
+  cudaEventRecord(g_prof.ev[2 * slot], st);
+}
+ProfScope::~ProfScope() {
+  if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
+}
 
 fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st);
 fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
@@ -79,6 +107,8 @@ static fsdit_status need(const void* p, const char* name) {
 }
 
 static size_t dsize(int dtype) { return dtype == FSDIT_BF16 ? 2 : 4; }
+// attention width: heads * head_dim (56 x 128 = 7168 next to hidden 5376)
+static int attn_dim(const fsdit_dims* d) { return d->heads * d->head_dim; }
 
 static fsdit_status check_dims(const fsdit_dims* d) {
   FS_TRY(need(d, "dims"));
@@ -86,9 +116,9 @@ static fsdit_status check_dims(const fsdit_dims* d) {
     set_error("dims.dtype %d is neither FSDIT_F32 nor FSDIT_BF16", d->dtype);
     return FSDIT_E_DTYPE;
   }
-  if (d->head_dim != 128 || d->heads <= 0 || d->hidden != d->heads * d->head_dim || d->hidden % 64 != 0 ||
+  if (d->head_dim != 128 || d->heads <= 0 || d->heads > 256 || d->hidden <= 0 || d->hidden % 64 != 0 ||
       d->hidden > 8192) {
-    set_error("dims: need head_dim 128, hidden = heads*128, hidden %% 64 == 0, hidden <= 8192 (got %d/%d/%d)",
+    set_error("dims: need head_dim 128, 0 < heads <= 256, hidden %% 64 == 0, hidden <= 8192 (got %d/%d/%d)",
               d->hidden, d->heads, d->head_dim);
     return FSDIT_E_SHAPE;
   }
@@ -118,7 +148,7 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.resid = resid;
   e.ldr = ldo;
   e.pos = pos;
-  e.rope_cols = 2 * d->hidden;
+  e.rope_cols = 2 * attn_dim(d);
   e.head_dim = d->head_dim;
   e.s0 = d->rope_split[0];
   e.s1 = d->rope_split[1];
@@ -129,14 +159,21 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
 fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep, int M, int N,
                            int K, cudaStream_t st) {
   if (M <= 0) return FSDIT_OK;
+  static const int cls_of[5] = {PC_GEMM_BIAS, PC_GEMM_BIAS_F32, PC_GEMM_QKV, PC_GEMM_GELU, PC_GEMM_RESID};
+  const double s = (double)dsize(d->dtype);
+  const double out_b = (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32) ? 4.0 : s;
+  const double by = ((double)M * K + (double)N * K) * s + (double)M * N * out_b +
+                    (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
+  ProfScope ps(cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);
   if (d->dtype == FSDIT_BF16) return launch_linear_tc(a, w, ep, M, N, K, st);
   return launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
 }
 
 fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n, cudaStream_t st) {
   if (n <= 0) return FSDIT_OK;
-  if (d->dtype == FSDIT_BF16) return launch_attention_tc(qkv, out, n, d->heads, d->hidden, st);
-  return launch_attention_simt(FSDIT_F32, qkv, out, n, d->heads, d->hidden, st);
+  ProfScope ps(PC_ATTN, 1, 4.0 * n * (double)n * attn_dim(d), 4.0 * n * (double)attn_dim(d) * dsize(d->dtype), st);
+  if (d->dtype == FSDIT_BF16) return launch_attention_tc(qkv, out, n, d->heads, attn_dim(d), st);
+  return launch_attention_simt(FSDIT_F32, qkv, out, n, d->heads, attn_dim(d), st);
 }
 
 // ---------------------------------------------------------------- workspace
@@ -153,8 +190,8 @@ struct Carve {
 struct BlockWs {
   float* xc;       // [n_c, hidden] compressed residual (compressed mode)
   int32_t* posc;   // [n_c, 3]
-  void* xn;        // [n, hidden] GEMM operand (normalized x / attention output)
-  void* qkv;       // [n, 3 hidden]
+  void* xn;        // [n, max(hidden, attn)] GEMM operand (normalized x / attention output)
+  void* qkv;       // [n, 3 attn]
   void* u;         // [n, ffn]
 };
 
@@ -163,8 +200,9 @@ static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, b
   const int n = compressed ? n_c : n_rows;
   w.xc = compressed ? (float*)c.take((size_t)n_c * d->hidden * 4) : nullptr;
   w.posc = compressed ? (int32_t*)c.take((size_t)n_c * 3 * 4) : nullptr;
-  w.xn = c.take((size_t)n * d->hidden * dsize(d->dtype));
-  w.qkv = c.take((size_t)n * 3 * d->hidden * dsize(d->dtype));
+  const int wide = d->hidden > attn_dim(d) ? d->hidden : attn_dim(d);
+  w.xn = c.take((size_t)n * wide * dsize(d->dtype));
+  w.qkv = c.take((size_t)n * 3 * attn_dim(d) * dsize(d->dtype));
   w.u = c.take((size_t)n * d->ffn * dsize(d->dtype));
   return w;
 }
@@ -173,12 +211,12 @@ static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, b
 // x[n, hidden] (fp32, in place): x += attn(...); x += ffn(...).
 static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
                                const int32_t* pos, int n, const BlockWs& ws, cudaStream_t st) {
-  const int H = d->hidden, F = d->ffn;
+  const int H = d->hidden, F = d->ffn, A = attn_dim(d);
   FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
-  FS_TRY(launch_linear(d, ws.xn, w->w_qkv, make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * H, nullptr, pos), n,
-                       3 * H, H, st));
+  FS_TRY(launch_linear(d, ws.xn, w->w_qkv, make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos), n,
+                       3 * A, H, st));
   FS_TRY(launch_attention(d, ws.qkv, ws.xn, n, st));
-  FS_TRY(launch_linear(d, ws.xn, w->w_o, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), n, H, H,
+  FS_TRY(launch_linear(d, ws.xn, w->w_o, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), n, H, A,
                        st));
   FS_TRY(launch_rmsnorm_cast(x_out, w->g_ffn, ws.xn, n, H, d->rms_eps, d->dtype, st));
   FS_TRY(launch_linear(d, ws.xn, w->w_1, make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr), n, F, H, st));
@@ -251,6 +289,58 @@ using namespace fsdit;
 extern "C" {
 
 const char* fsdit_last_error(void) { return t_err; }
+
+fsdit_status fsdit_profile_start(int max_launches) {
+  if (max_launches <= 0) {
+    set_error("profile: max_launches must be positive");
+    return FSDIT_E_SHAPE;
+  }
+  const size_t need_ev = 2 * (size_t)max_launches;
+  while (g_prof.ev.size() < need_ev) {
+    cudaEvent_t e;
+    FS_TRY(cuda_check(cudaEventCreate(&e), "cudaEventCreate"));
+    g_prof.ev.push_back(e);
+  }
+  g_prof.cls.assign(max_launches, 0);
+  g_prof.kernels.assign(max_launches, 0);
+  g_prof.flops.assign(max_launches, 0.0);
+  g_prof.bytes.assign(max_launches, 0.0);
+  g_prof.used = 0;
+  g_prof.on = true;
+  return FSDIT_OK;
+}
+
+int fsdit_profile_stop(fsdit_prof_entry* entries, int max_entries) {
+  g_prof.on = false;
+  if (g_prof.used == 0) return 0;
+  if (cuda_check(cudaEventSynchronize(g_prof.ev[2 * (g_prof.used - 1) + 1]), "cudaEventSynchronize") != FSDIT_OK)
+    return FSDIT_E_CUDA;
+  fsdit_prof_entry acc[PC_COUNT];
+  memset(acc, 0, sizeof(acc));
+  for (int i = 0; i < g_prof.used; ++i) {
+    float ms = 0.f;
+    if (cuda_check(cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]), "cudaEventElapsedTime") !=
+        FSDIT_OK)
+      return FSDIT_E_CUDA;
+    fsdit_prof_entry& e = acc[g_prof.cls[i]];
+    e.scopes += 1;
+    e.launches += g_prof.kernels[i];
+    e.ms += ms;
+    e.flops += g_prof.flops[i];
+    e.bytes += g_prof.bytes[i];
+  }
+  int n = 0;
+  for (int c = 0; c < PC_COUNT; ++c) {
+    if (acc[c].scopes == 0) continue;
+    if (entries != nullptr && n < max_entries) {
+      entries[n] = acc[c];
+      snprintf(entries[n].name, sizeof(entries[n].name), "%s", kProfNames[c]);
+    }
+    ++n;
+  }
+  g_prof.used = 0;
+  return n;
+}
 const char* fsdit_version(void) { return "fsdit 0.1 sm_100a"; }
 
 fsdit_status fsdit_device_error(fsdit_stream_t stream) {
@@ -296,8 +386,9 @@ static size_t stack_carve(Carve& c, const fsdit_dims* d, const fsdit_io_weights*
   BlockWs w;
   w.xc = comp ? (float*)c.take((size_t)n_c * d->hidden * 4) : nullptr;
   w.posc = comp ? (int32_t*)c.take((size_t)n_c * 3 * 4) : nullptr;
-  w.xn = c.take((size_t)N * d->hidden * dsize(d->dtype));
-  w.qkv = c.take((size_t)N * 3 * d->hidden * dsize(d->dtype));
+  const int wide = d->hidden > attn_dim(d) ? d->hidden : attn_dim(d);
+  w.xn = c.take((size_t)N * wide * dsize(d->dtype));
+  w.qkv = c.take((size_t)N * 3 * attn_dim(d) * dsize(d->dtype));
   w.u = c.take((size_t)N * d->ffn * dsize(d->dtype));
   *bw = w;
   return c.off;
@@ -393,8 +484,8 @@ fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, 
   if (epilogue == FSDIT_EPI_RESIDUAL) FS_TRY(need(resid, "resid"));
   if (epilogue == FSDIT_EPI_QKV_ROPE) {
     FS_TRY(need(pos, "pos"));
-    if (N != 3 * dims->hidden) {
-      set_error("linear: the RoPE epilogue needs N == 3*hidden");
+    if (N != 3 * attn_dim(dims)) {
+      set_error("linear: the RoPE epilogue needs N == 3*heads*head_dim");
       return FSDIT_E_SHAPE;
     }
   }

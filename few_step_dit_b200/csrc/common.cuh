@@ -138,6 +138,20 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
 
 // Host-side internal API shared by the .cu files.
 namespace fsdit {
+// Launch profiler: while fsdit_profile_start() is active, every launch scope
+// records a CUDA event pair on its stream plus the algorithmic FLOPs / bytes
+// of the work it launches (host arithmetic; nothing is read back until stop).
+enum ProfClass {
+  PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
+  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_COUNT
+};
+struct ProfScope {
+  ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);
+  ~ProfScope();
+  int slot;
+  cudaStream_t st;
+};
+
 int num_sms();
 void set_error(const char* fmt, ...);
 fsdit_status cuda_check(cudaError_t e, const char* what);
@@ -152,6 +166,6 @@ fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, i
                               cudaStream_t st);
 fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n, int heads,
                                    int hidden, cudaStream_t st);
-fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int hidden,
+fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int attn,
                                  cudaStream_t st);
 }  // namespace fsdit

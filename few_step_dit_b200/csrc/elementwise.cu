@@ -364,6 +364,7 @@ static int grid_for_rows(int rows, int per_sm) {
 fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st) {
   const int total = T * H * W;
   const int blocks = (total + 255) / 256;
+  ProfScope ps(PC_KEEPMAP, 1, 0.0, 4.0 * total + 4.0 * T * (H / 2 + 1) * (W / 2 + 1), st);
   keep_map_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(T, H, W, keep_idx, near_idx);
   return cuda_check(cudaGetLastError(), "keep_map_kernel");
 }
@@ -371,6 +372,7 @@ fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* ne
 fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
                            int n_keep, int n_grid, int n_rows, int hidden, cudaStream_t st) {
   const int n_out = n_keep + (n_rows - n_grid);
+  ProfScope ps(PC_GATHER, 1, 0.0, 8.0 * n_out * (double)hidden + (pos ? 24.0 * n_out : 0.0), st);
   gather_rows_kernel<<<grid_for_rows(n_out, 8), 256, 0, st>>>(x, pos, xc, posc, keep_idx, n_keep, n_grid, n_out,
                                                               hidden);
   return cuda_check(cudaGetLastError(), "gather_rows_kernel");
@@ -380,6 +382,8 @@ fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const
                               const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
                               cudaStream_t st) {
   const int g = grid_for_rows(n_rows, 8);
+  const double n_c = (double)n_keep + (n_rows - n_grid);
+  ProfScope ps(PC_BCAST, out != x ? 1 : 2, 0.0, ((double)n_grid + n_c + n_rows) * hidden * 4.0, st);
   if (out != x) {
     broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 0);
     return cuda_check(cudaGetLastError(), "broadcast_kernel");
@@ -394,6 +398,8 @@ fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
                                  cudaStream_t st) {
   const int grid = grid_for_rows(rows, 8);
+  const double s = dtype == FSDIT_BF16 ? 2.0 : 4.0;
+  ProfScope ps(PC_NORM, 1, 0.0, (double)rows * hidden * (4.0 + s) + hidden * s, st);
   if (dtype == FSDIT_BF16)
     rmsnorm_cast_kernel<bf16><<<grid, 256, 0, st>>>(x, (const bf16*)g, (bf16*)xn, rows, hidden, eps);
   else
@@ -408,6 +414,10 @@ static fsdit_status embed_t(float* x, int hidden, int row0, int rows, int kind, 
                             int ea, int eb, cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
   const int blocks = (rows + EMB_ROWS - 1) / EMB_ROWS;
+  ProfScope ps(PC_EMBED, 1, 2.0 * rows * (double)hidden * K,
+               (double)rows * hidden * 4.0 * (kind == 0 ? 2.0 : 1.0) + (double)rows * K * 4.0 +
+                   (double)hidden * K * sizeof(TW),
+               st);
   embed_kernel<TW><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in, (const TW*)b_in,
                                            text_proj, (const TW*)mod_emb, temb, modality, time_id, n_times, ea, eb);
   return cuda_check(cudaGetLastError(), "embed_kernel");
@@ -429,6 +439,8 @@ fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, in
                              cudaStream_t st) {
   const int blocks = num_sms() * 2;
   const size_t sm1 = (size_t)n_times * t_freq * sizeof(float);
+  ProfScope ps(PC_TIMEMLP, 2, 2.0 * n_times * (double)hidden * (t_freq + hidden),
+               (double)hidden * (t_freq + hidden) * (dtype == FSDIT_BF16 ? 2.0 : 4.0), st);
   Times8 times_dev;
   for (int i = 0; i < 8; ++i) times_dev.t[i] = i < n_times ? times_host[i] : 0.f;
   if (dtype == FSDIT_BF16) {
@@ -447,6 +459,10 @@ fsdit_status launch_heads(int dtype, const float* x, int row0, int rows, int hid
                           const void* b, int C, float eps, float* out, cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
   const int blocks = (rows + HEAD_ROWS - 1) / HEAD_ROWS;
+  ProfScope ps(PC_HEADS, 1, 2.0 * rows * (double)hidden * C,
+               (double)rows * hidden * 4.0 + (double)C * hidden * (dtype == FSDIT_BF16 ? 2.0 : 4.0) +
+                   (double)rows * C * 4.0,
+               st);
   if (dtype == FSDIT_BF16)
     heads_kernel<bf16><<<blocks, 256, 0, st>>>(x, row0, rows, hidden, (const bf16*)g, (const bf16*)w,
                                                (const bf16*)b, C, eps, out);
@@ -465,6 +481,7 @@ fsdit_status launch_euler(float* x, const float* v, const uint8_t* mod, const ui
   const size_t cap = (size_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) blocks = 1;
+  ProfScope ps(PC_EULER, 1, 2.0 * total, 12.0 * total + 2.0 * n_rows, st);
   euler_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, v, mod, mask, n_rows, width, c);
   return cuda_check(cudaGetLastError(), "euler_kernel");
 }

@@ -70,13 +70,13 @@ fsdit_status launch_linear_simt(int dtype, const void* a, const void* w, const E
 constexpr int SA_KEYS = 32;
 template <typename T>
 __global__ void __launch_bounds__(256) simt_attention_kernel(const T* __restrict__ qkv, T* __restrict__ out, int n,
-                                                             int hidden) {
+                                                             int attn) {
   __shared__ float Ks[SA_KEYS][128];
   __shared__ float Vs[SA_KEYS][128];
   const int head = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q_row = blockIdx.x * 8 + warp;
-  const size_t ld = (size_t)3 * hidden;
+  const size_t ld = (size_t)3 * attn;
   const float scale = rsqrtf(128.0f);
   float q[4], acc[4] = {0.f, 0.f, 0.f, 0.f};
   float m = -INFINITY, l = 0.f;
@@ -88,8 +88,8 @@ __global__ void __launch_bounds__(256) simt_attention_kernel(const T* __restrict
     for (int e = threadIdx.x; e < SA_KEYS * 128; e += blockDim.x) {
       const int r = e / 128, c = e % 128;
       const int j = j0 + r;
-      Ks[r][c] = (j < n) ? ld_f32<T>(qkv + (size_t)j * ld + hidden + head * 128 + c) : 0.f;
-      Vs[r][c] = (j < n) ? ld_f32<T>(qkv + (size_t)j * ld + 2 * hidden + head * 128 + c) : 0.f;
+      Ks[r][c] = (j < n) ? ld_f32<T>(qkv + (size_t)j * ld + attn + head * 128 + c) : 0.f;
+      Vs[r][c] = (j < n) ? ld_f32<T>(qkv + (size_t)j * ld + 2 * attn + head * 128 + c) : 0.f;
     }
     __syncthreads();
     const int nk = min(SA_KEYS, n - j0);
@@ -111,17 +111,17 @@ __global__ void __launch_bounds__(256) simt_attention_kernel(const T* __restrict
     const float inv = 1.0f / l;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      out[(size_t)q_row * hidden + head * 128 + lane * 4 + i] = cvt_from_f32<T>(acc[i] * inv);
+      out[(size_t)q_row * attn + head * 128 + lane * 4 + i] = cvt_from_f32<T>(acc[i] * inv);
   }
 }
 
-fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n, int heads, int hidden,
+fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n, int heads, int attn,
                                    cudaStream_t st) {
   dim3 grid((n + 7) / 8, heads);
   if (dtype == FSDIT_BF16)
-    simt_attention_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)qkv, (bf16*)out, n, hidden);
+    simt_attention_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)qkv, (bf16*)out, n, attn);
   else
-    simt_attention_kernel<float><<<grid, 256, 0, st>>>((const float*)qkv, (float*)out, n, hidden);
+    simt_attention_kernel<float><<<grid, 256, 0, st>>>((const float*)qkv, (float*)out, n, attn);
   return cuda_check(cudaGetLastError(), "simt_attention_kernel");
 }
 

@@ -57,6 +57,11 @@ class Tokens(C.Structure):
                 ("n_keep", C.c_int), ("near_idx", C.c_void_p)]
 
 
+class ProfEntry(C.Structure):
+    _fields_ = [("name", C.c_char * 32), ("scopes", C.c_int), ("launches", C.c_int),
+                ("ms", C.c_double), ("flops", C.c_double), ("bytes", C.c_double)]
+
+
 _P = C.c_void_p
 _I = C.c_int
 _F = C.c_float
@@ -65,6 +70,8 @@ _SIGS = {
     "fsdit_version": (C.c_char_p, []),
     "fsdit_device_error": (_I, [_P]),
     "fsdit_keep_count": (_I, [_I, _I, _I]),
+    "fsdit_profile_start": (_I, [_I]),
+    "fsdit_profile_stop": (_I, [C.POINTER(ProfEntry), _I]),
     "fsdit_block_workspace_size": (C.c_size_t, [C.POINTER(Dims), _I, _I]),
     "fsdit_stack_workspace_size": (C.c_size_t, [C.POINTER(Dims), C.POINTER(IOWeights),
                                                 C.POINTER(Tokens), _I]),
@@ -130,3 +137,18 @@ def ptr(t):
     if t is None:
         return None
     return C.c_void_p(t.data_ptr())
+
+
+def profile_start(max_launches=100000):
+    call("fsdit_profile_start", max_launches)
+
+
+def profile_stop():
+    """Per-class launch statistics recorded since profile_start()."""
+    lib = load()
+    buf = (ProfEntry * 32)()
+    n = lib.fsdit_profile_stop(buf, 32)
+    if n < 0:
+        check("fsdit_profile_stop", n)
+    return {buf[i].name.decode(): dict(scopes=buf[i].scopes, launches=buf[i].launches, ms=buf[i].ms,
+                                       flops=buf[i].flops, bytes=buf[i].bytes) for i in range(n)}

@@ -59,6 +59,10 @@ class Workload:
     rope_theta: float = 10000.0
 
     @property
+    def attn_dim(self):
+        return self.heads * self.head_dim
+
+    @property
     def n_video(self):
         T, H, W = self.grid
         return T * H * W
@@ -183,12 +187,12 @@ def _randn(shape, g, std, dtype, device):
 def make_block_weights(w: Workload, g: torch.Generator, device="cpu", dtype=None):
     """Raw block weights (Linear layout [out, in]) and RMSNorm gains."""
     dt = dtype or w.torch_dtype
-    H, F = w.hidden, w.ffn
+    H, F, A = w.hidden, w.ffn, w.attn_dim
     s = 0.02
     out = {
-        "w_qkv": _randn((3 * H, H), g, s, dt, device),
-        "b_qkv": _randn((3 * H,), g, s, dt, device),
-        "w_o": _randn((H, H), g, s, dt, device),
+        "w_qkv": _randn((3 * A, H), g, s, dt, device),
+        "b_qkv": _randn((3 * A,), g, s, dt, device),
+        "w_o": _randn((H, A), g, s, dt, device),
         "b_o": _randn((H,), g, s, dt, device),
         "w_1": _randn((F, H), g, s, dt, device),
         "b_1": _randn((F,), g, s, dt, device),

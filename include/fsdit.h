@@ -70,10 +70,12 @@ typedef enum { FSDIT_F32 = 0, FSDIT_BF16 = 1 } fsdit_dtype;
 enum { FSDIT_MOD_TEXT = 0, FSDIT_MOD_VIDEO = 1, FSDIT_MOD_AUDIO = 2, FSDIT_MOD_CONTROL = 3 };
 
 /* Model dimensions.  [tokendh] backbone section: hidden 5376, 56 heads of
- * 128, FFN 14336 (the Flash model keeps 42 of the 50 layers).  The head
- * dimension must be 128; rope_split gives the (t,h,w) chunk widths of a head
- * (32/48/48), each even, summing to head_dim.  hidden must be a multiple of 64
- * and equal heads*head_dim; ffn a multiple of 64. */
+ * 128, FFN 14336 (the Flash model keeps 42 of the 50 layers).  The heads span
+ * heads*head_dim channels (56 x 128 = 7168), which need not equal hidden: the
+ * qkv projection maps hidden -> 3*heads*head_dim and the output projection
+ * maps heads*head_dim -> hidden.  head_dim must be 128; rope_split gives the
+ * (t,h,w) chunk widths of a head (32/48/48), each even, summing to head_dim.
+ * hidden and ffn are multiples of 64, hidden <= 8192. */
 typedef struct {
   int hidden, heads, head_dim, ffn;
   int rope_split[3];
@@ -82,11 +84,11 @@ typedef struct {
   int dtype;        /* fsdit_dtype of weights and GEMM operands */
 } fsdit_dims;
 
-/* Weights of one pre-norm DiT block (all (device), `dtype`).
- *   w_qkv [3*hidden, hidden]  rows: q (hidden), k (hidden), v (hidden); head h
- *                             owns rows [h*128, h*128+128) of each part
- *   b_qkv [3*hidden]
- *   w_o   [hidden, hidden],  b_o [hidden]
+/* Weights of one pre-norm DiT block (all (device), `dtype`); A = heads*128.
+ *   w_qkv [3*A, hidden]  rows: q (A), k (A), v (A); head h owns rows
+ *                        [h*128, h*128+128) of each part
+ *   b_qkv [3*A]
+ *   w_o   [hidden, A],   b_o [hidden]
  *   w_1   [ffn, hidden],     b_1 [ffn]
  *   w_2   [hidden, ffn],     b_2 [hidden]
  *   g_attn, g_ffn [hidden]   RMSNorm gains */
@@ -137,6 +139,25 @@ FSDIT_API const char* fsdit_version(void);
  * reset gave up a bounded wait (and clears the word), else FSDIT_OK. */
 FSDIT_API fsdit_status fsdit_device_error(fsdit_stream_t stream);
 
+/* Launch profiler (measurement aid, off by default).  Between
+ * fsdit_profile_start(max_launches) and fsdit_profile_stop() every launch the
+ * library enqueues is bracketed by a CUDA event pair on its own stream (events
+ * are created once and reused).  stop() waits for the last event, then writes
+ * one entry per kernel class with its launches, summed device time and the
+ * algorithmic FLOPs and bytes of those launches (computed on the host from the
+ * shapes), and returns the number of classes (negative fsdit_status on error).
+ * Not thread-safe; launches beyond max_launches are not recorded. */
+typedef struct {
+  char name[32];
+  int scopes;   /* launch scopes recorded */
+  int launches; /* kernels launched inside them */
+  double ms;    /* summed device time */
+  double flops; /* algorithmic FLOPs */
+  double bytes; /* algorithmic bytes moved */
+} fsdit_prof_entry;
+FSDIT_API fsdit_status fsdit_profile_start(int max_launches);
+FSDIT_API int fsdit_profile_stop(fsdit_prof_entry* entries, int max_entries);
+
 /* Number of kept tokens of a T x H x W grid: T * (H/2+1) * (W/2+1). */
 FSDIT_API int fsdit_keep_count(int T, int H, int W);
 
@@ -186,8 +207,9 @@ FSDIT_API fsdit_status fsdit_rmsnorm_cast(const float* x, const void* g, void* x
 /* Epilogues of fsdit_linear (all add the bias first):
  *   FSDIT_EPI_BIAS       out (dtype)  = acc + b
  *   FSDIT_EPI_BIAS_F32   out (f32)    = acc + b
- *   FSDIT_EPI_QKV_ROPE   out (dtype)  = rope(acc + b) on columns < 2*hidden
- *                        (q and k), per row position pos[row]
+ *   FSDIT_EPI_QKV_ROPE   out (dtype)  = rope(acc + b) on columns < 2*heads*128
+ *                        (q and k; N must be 3*heads*128), per row position
+ *                        pos[row]
  *   FSDIT_EPI_GELU       out (dtype)  = gelu_tanh(acc + b)
  *   FSDIT_EPI_RESIDUAL   out (f32)    = resid + acc + b   (out may equal resid) */
 enum {
@@ -209,8 +231,9 @@ FSDIT_API fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const
 
 /* Joint attention ([tokendh] backbone section: one sequence of text,
  * video and audio tokens through one denoiser): for each head,
- * softmax(q k^T / sqrt(128)) v over all n rows, no mask.  qkv [n, 3*hidden]
- * in `dtype` (q | k | v, RoPE already applied); out [n, hidden] in `dtype`. */
+ * softmax(q k^T / sqrt(128)) v over all n rows, no mask.  With A = heads*128:
+ * qkv [n, 3*A] in `dtype` (q | k | v, RoPE already applied); out [n, A] in
+ * `dtype`. */
 FSDIT_API fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n,
                              fsdit_stream_t stream);
 

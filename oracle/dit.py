@@ -190,16 +190,20 @@ def dit_block(x, w, pos, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
 
     h = x + Wo . attn(rope(q), rope(k), v) + bo, with [q k v] = Wqkv . rmsnorm(x) + b;
     y = h + W2 . gelu_tanh(W1 . rmsnorm(h) + b1) + b2.
+    [tokendh, backbone section] gives hidden 5376 and 56 heads of 128: the
+    heads span 56 x 128 = 7168 channels, so q, k, v are each heads*head_dim
+    wide (Wqkv is [3*heads*head_dim, H]) and Wo maps them back to H.
     Reading: pre-RMSNorm with a learned gain, biases on every projection,
     RoPE on q and k at each token's own (t, h, w) position.
     """
     x = np.asarray(x, dtype=F64)
-    n, H = x.shape
+    n = x.shape[0]
+    A = heads * head_dim          # attention width; 56 x 128 = 7168 next to hidden 5376
     xn = rms_norm(x, w["g_attn"], eps)
     qkv = linear(xn, w["w_qkv"], w["b_qkv"])
-    q = qkv[:, 0 * H:1 * H].reshape(n, heads, head_dim)
-    k = qkv[:, 1 * H:2 * H].reshape(n, heads, head_dim)
-    v = qkv[:, 2 * H:3 * H].reshape(n, heads, head_dim)
+    q = qkv[:, 0 * A:1 * A].reshape(n, heads, head_dim)
+    k = qkv[:, 1 * A:2 * A].reshape(n, heads, head_dim)
+    v = qkv[:, 2 * A:3 * A].reshape(n, heads, head_dim)
     q = apply_rope(q, pos, rope_split, theta)
     k = apply_rope(k, pos, rope_split, theta)
     a = attention(q, k, v)

@@ -96,6 +96,17 @@ def test_bf16_block_small_width(grid, compress):
     assert O.rel_l2(got - x, ref - x) < 1e-2
 
 
+@pytest.mark.parametrize("dtype,bound", [("f32", 1e-5), ("bf16", 1e-2)])
+def test_block_attention_width_differs_from_hidden(dtype, bound):
+    # 3 heads of 128 = 384 attention channels next to hidden 256 (the full
+    # model has 56 x 128 = 7168 next to 5376)
+    w = S.scaled(S.WORKLOADS["tiny_block_f32"], heads=3, dtype=dtype)
+    assert w.attn_dim != w.hidden
+    got, ref, x = _block_case(w, True)
+    assert O.rel_l2(got, ref) < bound
+    assert O.rel_l2(got - x, ref - x) < bound
+
+
 def test_tiny_fp32_euler_step_from_block_velocity():
     # one Euler step video 0.2 -> 0.0769, audio 0.5 -> 0.25 on the tiny workload
     w = S.WORKLOADS["tiny_block_f32"]
