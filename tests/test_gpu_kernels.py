@@ -189,6 +189,26 @@ def test_attention(dtype, n, heads):
     assert err < (1e-5 if dtype == torch.float32 else 1e-2), err
 
 
+@pytest.mark.parametrize("n,heads,check_heads", [(3668, 56, (0, 17, 55)), (12560, 56, (3, 42))])
+def test_attention_full_size_sampled_heads(n, heads, check_heads):
+    # the Flash sequence lengths (compressed and full) at the 56-head width;
+    # the oracle runs on a few heads, the kernel on all of them
+    g = _rng(8)
+    A = heads * 128
+    dims = api.make_dims(5376, heads, 14336, torch.bfloat16)
+    qkv = (torch.randn(n, 3 * A, generator=g) * 1.5).bfloat16()
+    out = api.attention(dims, qkv.to(DEV))
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    for h in check_heads:
+        q = qkv[:, h * 128:(h + 1) * 128].double().numpy()[:, None, :]
+        k = qkv[:, A + h * 128:A + (h + 1) * 128].double().numpy()[:, None, :]
+        v = qkv[:, 2 * A + h * 128:2 * A + (h + 1) * 128].double().numpy()[:, None, :]
+        ref = O.attention(q, k, v)
+        err = O.rel_l2(got[:, h * 128:(h + 1) * 128], ref)
+        assert err < 1e-2, (h, err)
+
+
 # ---------------------------------------------------------------- Euler
 
 
