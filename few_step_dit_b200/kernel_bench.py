@@ -1,0 +1,109 @@
+"""Time single hot-path kernels through the C ABI (CUDA events, warm).
+
+Examples:
+  python -m few_step_dit_b200.kernel_bench attention --n 12560 --heads 56
+  python -m few_step_dit_b200.kernel_bench gemm --M 12560 --N 21504 --K 5376 --epi qkv
+  python -m few_step_dit_b200.kernel_bench block --workload flash_block_6x34x60
+Inputs are seeded Gaussians; each case prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from few_step_dit_b200 import api, build as B, lib as L  # noqa: E402
+from few_step_dit_b200 import synthetic as S  # noqa: E402
+
+EPI = {"bias": L.EPI_BIAS, "bias_f32": L.EPI_BIAS_F32, "qkv": L.EPI_QKV_ROPE, "gelu": L.EPI_GELU,
+       "residual": L.EPI_RESIDUAL}
+
+
+def time_it(fn, iters, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    e.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def case_attention(a):
+    g = torch.Generator(device="cuda").manual_seed(1)
+    A = a.heads * 128
+    dims = api.make_dims(5376, a.heads, 14336, L.BF16)
+    qkv = torch.randn(a.n, 3 * A, generator=g, device="cuda").mul_(1.5).bfloat16()
+    out = torch.empty(a.n, A, dtype=torch.bfloat16, device="cuda")
+    ms = time_it(lambda: api.attention(dims, qkv, out), a.iters, a.warmup)
+    fl = 4.0 * a.n * a.n * A
+    return {"case": "attention", "n": a.n, "heads": a.heads, "ms": ms, "tflops": fl / ms / 1e9}
+
+
+def case_gemm(a):
+    g = torch.Generator(device="cuda").manual_seed(2)
+    epi = EPI[a.epi]
+    heads = a.N // 3 // 128 if epi == L.EPI_QKV_ROPE else 56
+    dims = api.make_dims(5376, heads, 14336, L.BF16)
+    x = torch.randn(a.M, a.K, generator=g, device="cuda").bfloat16()
+    w = torch.randn(a.N, a.K, generator=g, device="cuda").mul_(0.02).bfloat16()
+    b = torch.randn(a.N, generator=g, device="cuda").mul_(0.02).bfloat16()
+    resid = torch.randn(a.M, a.N, generator=g, device="cuda") if epi == L.EPI_RESIDUAL else None
+    pos = torch.randint(0, 60, (a.M, 3), generator=g, device="cuda", dtype=torch.int32) \
+        if epi == L.EPI_QKV_ROPE else None
+    od = torch.float32 if epi in (L.EPI_RESIDUAL, L.EPI_BIAS_F32) else torch.bfloat16
+    out = torch.empty(a.M, a.N, dtype=od, device="cuda")
+    ms = time_it(lambda: api.linear(dims, x, w, b, epi, resid=resid, pos=pos, out=out), a.iters, a.warmup)
+    fl = 2.0 * a.M * a.N * a.K
+    return {"case": "gemm", "M": a.M, "N": a.N, "K": a.K, "epi": a.epi, "ms": ms, "tflops": fl / ms / 1e9}
+
+
+def case_block(a):
+    w = S.WORKLOADS[a.workload]
+    layers, _ = S.make_weights(w, device="cuda", n_layers=1)
+    tags = S.pack_tokens(w)
+    seq = api.Sequence.from_workload(w, tags, "cuda", compress=True)
+    bw = api.BlockWeights(layers[0])
+    dims = api.dims_of(w)
+    x = torch.randn(w.n_tokens, w.hidden, device="cuda")
+    out = torch.empty_like(x)
+    res = {"case": "block", "workload": a.workload, "tokens": w.n_tokens, "kept": seq.n_keep}
+    for comp in (True, False):
+        ms = time_it(lambda: api.block_forward(dims, bw, seq, x, out, compress=comp), a.iters, a.warmup)
+        res["ms_compressed" if comp else "ms_full"] = ms
+    return res
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("case", choices=["attention", "gemm", "block"])
+    p.add_argument("--n", type=int, default=12560)
+    p.add_argument("--heads", type=int, default=56)
+    p.add_argument("--M", type=int, default=12560)
+    p.add_argument("--N", type=int, default=21504)
+    p.add_argument("--K", type=int, default=5376)
+    p.add_argument("--epi", default="qkv", choices=sorted(EPI))
+    p.add_argument("--workload", default="flash_block_6x34x60")
+    p.add_argument("--iters", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    a = p.parse_args()
+    B.build()
+    L.load()
+    res = {"attention": case_attention, "gemm": case_gemm, "block": case_block}[a.case](a)
+    api.device_error()
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
