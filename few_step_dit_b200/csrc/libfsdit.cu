@@ -5,3 +5,4 @@
 #include "simt.cu"
 #include "gemm_tc.cu"
 #include "attn_tc.cu"
+#include "noalloc.cu"

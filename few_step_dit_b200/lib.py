@@ -83,6 +83,8 @@ _SIGS = {
     "fsdit_attention": (_I, [C.POINTER(Dims), _P, _P, _I, _P]),
     "dit_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), C.POINTER(Tokens), _P, _P,
                                _P, C.c_size_t, _P]),
+    "dit_block_forward_noalloc": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), C.POINTER(Tokens),
+                                       _P, _P, _P]),
     "dit_stack_forward": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(C.c_uint8),
                                C.POINTER(IOWeights), C.POINTER(Tokens), C.POINTER(_F), _I, _P, _P,
                                _P, _P, _P, _P, C.c_size_t, _P]),

@@ -291,6 +291,31 @@ FSDIT_API fsdit_status dit_flow_sample(const fsdit_dims* dims, int n_layers,
                              const void* text_emb, float* audio_lat, void* workspace,
                              size_t ws_bytes, fsdit_stream_t stream);
 
+/* The paper has no counterpart to this entry point; it exists for callers of
+ * this library that cannot call cudaMalloc -- for example a host application
+ * whose device memory is owned by its own pool allocator, or a plain C caller
+ * that must not allocate after start-up -- and so cannot provide the
+ * workspace dit_block_forward needs.
+ *
+ * Same computation and arguments as dit_block_forward, minus the workspace:
+ * the scratch comes from one static device array of 32 MiB inside the
+ * library (every GPU that loads libfsdit.so holds it until the process
+ * exits).  The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine.  Returns FSDIT_E_WORKSPACE, launching nothing, when the
+ * block's scratch (fsdit_block_workspace_size) exceeds 32 MiB -- in bf16
+ * about 390 tokens at hidden 5376 / 56 heads, about 10,900 at hidden 256 /
+ * 2 heads.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array and it keeps the last call's
+ * contents (nothing in it needs to start at zero: every buffer is written
+ * before it is read).  Calls that overlap on the GPU -- on different streams,
+ * or from different threads -- race on it; serialize them. */
+FSDIT_API fsdit_status dit_block_forward_noalloc(const fsdit_dims* dims, const fsdit_block_weights* w,
+                                                 const fsdit_tokens* tok, const float* x_in, float* x_out,
+                                                 fsdit_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
