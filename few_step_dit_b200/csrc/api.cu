@@ -15,7 +15,7 @@ namespace fsdit {
 static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "gemm_gelu", "gemm_bias_f32",
                                            "gemm_bias",     "attention",     "rmsnorm_cast", "gather",
                                            "broadcast",     "embed",         "time_mlp",  "heads",
-                                           "euler",         "keep_map"};
+                                           "euler",         "keep_map",  "rope_table"};
 struct Prof {
   bool on = false;
   int used = 0;
@@ -53,8 +53,8 @@ fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, i
 fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, int t_freq, const void* w1,
                              const void* b1, const void* w2, const void* b2, float* h1, float* temb, int hidden,
                              cudaStream_t st);
-fsdit_status launch_heads(int dtype, const float* x, int row0, int rows, int hidden, const void* g, const void* w,
-                          const void* b, int C, float eps, float* out, cudaStream_t st);
+fsdit_status launch_rope_table(const int32_t* pos, int rows, int head_dim, int s0, int s1, float log2_theta,
+                               float2* cs, cudaStream_t st);
 fsdit_status launch_euler(float* x, const float* v, const uint8_t* mod, const uint8_t* mask, int n_rows, int width,
                           const float* t_cur, const float* t_next, cudaStream_t st);
 
@@ -148,6 +148,7 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.resid = resid;
   e.ldr = ldo;
   e.pos = pos;
+  e.rope_cs = nullptr;
   e.rope_cols = 2 * attn_dim(d);
   e.head_dim = d->head_dim;
   e.s0 = d->rope_split[0];
@@ -157,14 +158,14 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
 }
 
 fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep, int M, int N,
-                           int K, cudaStream_t st) {
+                           int K, cudaStream_t st, int prof_cls) {
   if (M <= 0) return FSDIT_OK;
   static const int cls_of[5] = {PC_GEMM_BIAS, PC_GEMM_BIAS_F32, PC_GEMM_QKV, PC_GEMM_GELU, PC_GEMM_RESID};
   const double s = (double)dsize(d->dtype);
   const double out_b = (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32) ? 4.0 : s;
   const double by = ((double)M * K + (double)N * K) * s + (double)M * N * out_b +
                     (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
-  ProfScope ps(cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);
+  ProfScope ps(prof_cls >= 0 ? prof_cls : cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);
   if (d->dtype == FSDIT_BF16) return launch_linear_tc(a, w, ep, M, N, K, st);
   return launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
 }
@@ -193,6 +194,8 @@ struct BlockWs {
   void* xn;        // [n, max(hidden, attn)] GEMM operand (normalized x / attention output)
   void* qkv;       // [n, 3 attn]
   void* u;         // [n, ffn]
+  float2* rope;    // [n, head_dim/2] (cos, sin) table of the rows' positions
+  float2* rope_c;  // stack only: table of the compressed rows
 };
 
 static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, bool compressed) {
@@ -204,17 +207,25 @@ static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, b
   w.xn = c.take((size_t)n * wide * dsize(d->dtype));
   w.qkv = c.take((size_t)n * 3 * attn_dim(d) * dsize(d->dtype));
   w.u = c.take((size_t)n * d->ffn * dsize(d->dtype));
+  w.rope = (float2*)c.take((size_t)n * (d->head_dim / 2) * sizeof(float2));
+  w.rope_c = nullptr;
   return w;
 }
 
 // ---------------------------------------------------------------- block body
 // x[n, hidden] (fp32, in place): x += attn(...); x += ffn(...).
+static fsdit_status rope_table(const fsdit_dims* d, const int32_t* pos, int rows, float2* cs, cudaStream_t st) {
+  return launch_rope_table(pos, rows, d->head_dim, d->rope_split[0], d->rope_split[1], log2f(d->rope_theta), cs, st);
+}
+
+// x_in -> x_out over n rows; `rope` is the (cos, sin) table of the rows' positions.
 static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
-                               const int32_t* pos, int n, const BlockWs& ws, cudaStream_t st) {
+                               const int32_t* pos, const float2* rope, int n, const BlockWs& ws, cudaStream_t st) {
   const int H = d->hidden, F = d->ffn, A = attn_dim(d);
   FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
-  FS_TRY(launch_linear(d, ws.xn, w->w_qkv, make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos), n,
-                       3 * A, H, st));
+  EpiParams qkv_ep = make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos);
+  qkv_ep.rope_cs = rope;
+  FS_TRY(launch_linear(d, ws.xn, w->w_qkv, qkv_ep, n, 3 * A, H, st));
   FS_TRY(launch_attention(d, ws.qkv, ws.xn, n, st));
   FS_TRY(launch_linear(d, ws.xn, w->w_o, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), n, H, A,
                        st));
@@ -390,6 +401,8 @@ static size_t stack_carve(Carve& c, const fsdit_dims* d, const fsdit_io_weights*
   w.xn = c.take((size_t)N * wide * dsize(d->dtype));
   w.qkv = c.take((size_t)N * 3 * attn_dim(d) * dsize(d->dtype));
   w.u = c.take((size_t)N * d->ffn * dsize(d->dtype));
+  w.rope = (float2*)c.take((size_t)N * (d->head_dim / 2) * sizeof(float2));
+  w.rope_c = comp ? (float2*)c.take((size_t)n_c * (d->head_dim / 2) * sizeof(float2)) : nullptr;
   *bw = w;
   return c.off;
 }
@@ -524,9 +537,13 @@ fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_block_weights
     set_error("workspace: need %zu bytes, got %zu", c.off, ws_bytes);
     return FSDIT_E_WORKSPACE;
   }
-  if (!comp) return block_body(dims, w, const_cast<float*>(x_in), x_out, tok->pos_thw, n, ws, st);
+  if (!comp) {
+    FS_TRY(rope_table(dims, tok->pos_thw, n, ws.rope, st));
+    return block_body(dims, w, const_cast<float*>(x_in), x_out, tok->pos_thw, ws.rope, n, ws, st);
+  }
   FS_TRY(launch_gather(x_in, tok->pos_thw, ws.xc, ws.posc, tok->keep_idx, tok->n_keep, n_grid, n, dims->hidden, st));
-  FS_TRY(block_body(dims, w, ws.xc, ws.xc, ws.posc, n_c, ws, st));
+  FS_TRY(rope_table(dims, ws.posc, n_c, ws.rope, st));
+  FS_TRY(block_body(dims, w, ws.xc, ws.xc, ws.posc, ws.rope, n_c, ws, st));
   if (x_out != x_in) {
     FS_TRY(launch_broadcast(x_in, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, n, dims->hidden, st));
   } else {
@@ -543,9 +560,10 @@ static fsdit_status check_io(const fsdit_dims* d, const fsdit_io_weights* io) {
   const char* names[] = {"w_vin", "b_vin", "w_tin", "b_tin", "w_ain", "b_ain", "mod_emb", "w_t1",
                          "b_t1",  "w_t2",  "b_t2",  "g_out", "w_vout", "b_vout", "w_aout", "b_aout"};
   for (int i = 0; i < 16; ++i) FS_TRY(need(ptrs[i], names[i]));
-  if (io->c_video <= 0 || io->c_video > 64 || io->c_audio <= 0 || io->c_audio > 64 || io->c_text <= 0 ||
-      io->c_text % 8 != 0 || io->t_freq <= 0 || io->t_freq % 2 != 0 || io->t_freq > 1024) {
-    set_error("io: need 0 < c_video, c_audio <= 64, c_text %% 8 == 0, even t_freq <= 1024");
+  if (io->c_video <= 0 || io->c_video > 64 || io->c_video % 4 != 0 || io->c_audio <= 0 || io->c_audio > 64 ||
+      io->c_audio % 4 != 0 || io->c_text <= 0 || io->c_text % 8 != 0 || io->t_freq <= 0 || io->t_freq % 2 != 0 ||
+      io->t_freq > 1024) {
+    set_error("io: need c_video, c_audio in (0, 64] and multiples of 4, c_text %% 8 == 0, even t_freq <= 1024");
     return FSDIT_E_SHAPE;
   }
   (void)d;
@@ -585,25 +603,40 @@ static fsdit_status stack_forward_impl(const fsdit_dims* dims, int n_layers, con
   const int N = tok->n_tokens;
   const int n_grid = tok->grid_t * tok->grid_h * tok->grid_w;
   const int n_c = tok->keep_idx ? n_compressed(tok) : N;
+  bool have_full_rope = false, have_comp_rope = false;
   int l = 0;
   while (l < n_layers) {
     if (!layer_compress[l] || tok->keep_idx == nullptr) {
-      FS_TRY(block_body(dims, &layers[l], x, x, tok->pos_thw, N, bw, st));
+      if (!have_full_rope) {
+        FS_TRY(rope_table(dims, tok->pos_thw, N, bw.rope, st));
+        have_full_rope = true;
+      }
+      FS_TRY(block_body(dims, &layers[l], x, x, tok->pos_thw, bw.rope, N, bw, st));
       ++l;
       continue;
     }
     FS_TRY(launch_gather(x, tok->pos_thw, bw.xc, bw.posc, tok->keep_idx, tok->n_keep, n_grid, N, H, st));
+    if (!have_comp_rope) {
+      FS_TRY(rope_table(dims, bw.posc, n_c, bw.rope_c, st));
+      have_comp_rope = true;
+    }
     while (l < n_layers && layer_compress[l]) {
-      FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, n_c, bw, st));
+      FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, bw.rope_c, n_c, bw, st));
       ++l;
     }
     FS_TRY(launch_broadcast(x, bw.xc, x, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, N, H, st));
   }
-  // heads
-  FS_TRY(launch_heads(dims->dtype, x, 0, tok->n_vrows, H, io->g_out, io->w_vout, io->b_vout, io->c_video,
-                      dims->rms_eps, v_video, st));
-  FS_TRY(launch_heads(dims->dtype, x, tok->n_vrows + tok->n_text, tok->n_audio, H, io->g_out, io->w_aout, io->b_aout,
-                      io->c_audio, dims->rms_eps, v_audio, st));
+  // heads: final RMSNorm into the GEMM operand buffer, then the two projections
+  FS_TRY(launch_rmsnorm_cast(x, io->g_out, bw.xn, N, H, dims->rms_eps, dims->dtype, st));
+  if (tok->n_vrows > 0) {
+    EpiParams ep = make_ep(dims, FSDIT_EPI_BIAS_F32, io->b_vout, v_video, io->c_video, nullptr, nullptr);
+    FS_TRY(launch_linear(dims, bw.xn, io->w_vout, ep, tok->n_vrows, io->c_video, H, st, PC_HEADS));
+  }
+  if (tok->n_audio > 0) {
+    const uint8_t* xa = (const uint8_t*)bw.xn + (size_t)(tok->n_vrows + tok->n_text) * H * dsize(dims->dtype);
+    EpiParams ep = make_ep(dims, FSDIT_EPI_BIAS_F32, io->b_aout, v_audio, io->c_audio, nullptr, nullptr);
+    FS_TRY(launch_linear(dims, xa, io->w_aout, ep, tok->n_audio, io->c_audio, H, st, PC_HEADS));
+  }
   return FSDIT_OK;
 }
 

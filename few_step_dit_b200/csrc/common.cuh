@@ -62,6 +62,7 @@ struct EpiParams {
   const float* resid;   // [M, ldr] (FSDIT_EPI_RESIDUAL)
   int ldr;
   const int32_t* pos;   // [M][3] (FSDIT_EPI_QKV_ROPE)
+  const float2* rope_cs;  // [M][head_dim/2] (cos, sin) per pair, or null: compute from pos
   int rope_cols;        // columns [0, rope_cols) are rotated
   int head_dim, s0, s1;
   float log2_theta;
@@ -76,11 +77,23 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
   for (int i = 0; i < CNT; ++i) v[i] += ld_f32<TW>(bias + col + i);
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
     if (col < p.rope_cols) {
-      const int32_t* pos3 = p.pos + (size_t)row * 3;
+      if (p.rope_cs != nullptr) {
+        // CNT consecutive columns of one head: pairs (col % head_dim)/2 ..
+        const float2* cs = p.rope_cs + (size_t)row * (p.head_dim >> 1) + ((col % p.head_dim) >> 1);
 #pragma unroll
-      for (int i = 0; i < CNT; i += 2) {
-        int d = (col + i) % p.head_dim;
-        rope_pair(v[i], v[i + 1], d, p.s0, p.s1, p.head_dim, pos3, p.log2_theta);
+        for (int i = 0; i < CNT; i += 2) {
+          const float2 t = cs[i >> 1];
+          const float a = v[i], b = v[i + 1];
+          v[i] = a * t.x - b * t.y;
+          v[i + 1] = a * t.y + b * t.x;
+        }
+      } else {
+        const int32_t* pos3 = p.pos + (size_t)row * 3;
+#pragma unroll
+        for (int i = 0; i < CNT; i += 2) {
+          int d = (col + i) % p.head_dim;
+          rope_pair(v[i], v[i + 1], d, p.s0, p.s1, p.head_dim, pos3, p.log2_theta);
+        }
       }
     }
   } else if (p.epi == FSDIT_EPI_GELU) {
@@ -143,7 +156,7 @@ namespace fsdit {
 // of the work it launches (host arithmetic; nothing is read back until stop).
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
-  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_COUNT
+  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);
@@ -157,7 +170,7 @@ void set_error(const char* fmt, ...);
 fsdit_status cuda_check(cudaError_t e, const char* what);
 
 fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep,
-                           int M, int N, int K, cudaStream_t st);
+                           int M, int N, int K, cudaStream_t st, int prof_cls = -1);
 fsdit_status launch_linear_simt(int dtype, const void* a, const void* w, const EpiParams& ep,
                                 int M, int N, int K, cudaStream_t st);
 fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep, int M, int N,

@@ -159,6 +159,22 @@ __global__ void __launch_bounds__(256) rmsnorm_cast_kernel(const float* __restri
   }
 }
 
+// ---------------------------------------------------------------- RoPE table
+// cs[r][j] = (cos, sin) of the angle of pair j of a head for row r; the QKV
+// epilogue reads it instead of evaluating sincos per element.  Positions are
+// constant across layers and evaluations, so one table serves a whole pass.
+__global__ void rope_table_kernel(const int32_t* __restrict__ pos, int rows, int head_dim, int s0, int s1,
+                                  float log2_theta, float2* __restrict__ cs) {
+  const int pairs = head_dim >> 1;
+  const size_t total = (size_t)rows * pairs;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / pairs), j = (int)(i % pairs);
+    float a = 1.0f, b = 0.0f;  // rotating (1, 0) yields (cos, sin)
+    rope_pair(a, b, 2 * j, s0, s1, head_dim, pos + (size_t)r * 3, log2_theta);
+    cs[i] = make_float2(a, b);
+  }
+}
+
 // ---------------------------------------------------------------- embedding
 // x[r] = src(r) + mod_emb[modality[r]] + temb[time_id[r]], where src(r) is the
 // small-K projection lat[r'] W^T + b of a video/control or audio row, or the
@@ -168,7 +184,7 @@ __global__ void __launch_bounds__(256) rmsnorm_cast_kernel(const float* __restri
 constexpr int EMB_ROWS = 16;
 constexpr int EMB_MAXK = 64;
 
-template <typename TW>
+template <typename TW, int KMAX>
 __global__ void __launch_bounds__(256) embed_kernel(
     float* __restrict__ x, int hidden, int row0, int rows, int kind,  // kind: 0 text, 1 latent
     const float* __restrict__ lat, int K, const TW* __restrict__ w_in, const TW* __restrict__ b_in,
@@ -192,24 +208,26 @@ __global__ void __launch_bounds__(256) embed_kernel(
     s_tid[threadIdx.x] = t;
   }
   if (kind == 1) {
-    for (int i = threadIdx.x; i < nr * K; i += blockDim.x)
-      s_lat[i / K][i % K] = lat[(size_t)(rb0 + i / K) * K + (i % K)];
+    for (int i = threadIdx.x; i < EMB_ROWS * KMAX; i += blockDim.x) {
+      const int rr = i / KMAX, kk = i % KMAX;
+      s_lat[rr][kk] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
+    }
   }
   __syncthreads();
   for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
-    float wr[EMB_MAXK];
+    float wr[KMAX];  // one weight row in registers (KMAX is a compile-time bound on K)
     float bias = 0.f;
     if (kind == 1) {
-#pragma unroll 8
-      for (int k = 0; k < K; ++k) wr[k] = ld_f32<TW>(w_in + (size_t)c * K + k);
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) wr[k] = k < K ? ld_f32<TW>(w_in + (size_t)c * K + k) : 0.f;
       bias = ld_f32<TW>(b_in + c);
     }
     for (int j = 0; j < nr; ++j) {
       float acc;
       if (kind == 1) {
         acc = bias;
-#pragma unroll 8
-        for (int k = 0; k < K; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
       } else {
         acc = text_proj[(size_t)(rb0 + j) * hidden + c];
       }
@@ -278,67 +296,6 @@ __global__ void time_mlp2_kernel(const float* __restrict__ h1, int n_times, cons
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
       if (lane == 0 && t < n_times) temb[(size_t)t * hidden + c] = a + ld_f32<TW>(b2 + c);
-    }
-  }
-}
-
-// ---------------------------------------------------------------- output heads
-// v[r, c] = rstd_r * sum_k x[r,k] g[k] W[c,k] + b[c] for C <= 64 outputs.  A
-// block owns HEAD_ROWS rows; x and g*W are staged in shared memory in chunks
-// of HEAD_KC channels; the row sum of squares is accumulated on the way.
-constexpr int HEAD_ROWS = 64;
-constexpr int HEAD_KC = 64;
-constexpr int HEAD_MAXC = 64;
-template <typename TW>
-__global__ void __launch_bounds__(256) heads_kernel(const float* __restrict__ x, int row0, int rows, int hidden,
-                                                    const TW* __restrict__ g, const TW* __restrict__ w,
-                                                    const TW* __restrict__ b, int C, float eps,
-                                                    float* __restrict__ out) {
-  __shared__ float s_x[HEAD_ROWS][HEAD_KC + 1];
-  __shared__ float s_w[HEAD_MAXC][HEAD_KC + 1];
-  __shared__ float s_ss[HEAD_ROWS];
-  const int rb = blockIdx.x * HEAD_ROWS;
-  const int nr = min(HEAD_ROWS, rows - rb);
-  if (nr <= 0) return;
-  // thread -> (row j, output group): 256 threads = 64 rows x 4 groups of C/4 outputs
-  const int j = threadIdx.x >> 2, grp = threadIdx.x & 3;
-  const int per = (C + 3) / 4;
-  float acc[HEAD_MAXC / 4];
-#pragma unroll
-  for (int i = 0; i < HEAD_MAXC / 4; ++i) acc[i] = 0.f;
-  float ss = 0.f;
-  for (int k0 = 0; k0 < hidden; k0 += HEAD_KC) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < HEAD_ROWS * HEAD_KC; i += blockDim.x) {
-      const int rr = i / HEAD_KC, kk = i % HEAD_KC;
-      s_x[rr][kk] = (rr < nr) ? x[(size_t)(row0 + rb + rr) * hidden + k0 + kk] : 0.f;
-    }
-    for (int i = threadIdx.x; i < C * HEAD_KC; i += blockDim.x) {
-      const int cc = i / HEAD_KC, kk = i % HEAD_KC;
-      s_w[cc][kk] = ld_f32<TW>(w + (size_t)cc * hidden + k0 + kk) * ld_f32<TW>(g + k0 + kk);
-    }
-    __syncthreads();
-    if (grp == 0) {
-      for (int kk = 0; kk < HEAD_KC; ++kk) ss = fmaf(s_x[j][kk], s_x[j][kk], ss);
-    }
-#pragma unroll
-    for (int i = 0; i < HEAD_MAXC / 4; ++i) {
-      const int cc = grp * per + i;
-      if (i < per && cc < C) {
-        float a = acc[i];
-        for (int kk = 0; kk < HEAD_KC; ++kk) a = fmaf(s_x[j][kk], s_w[cc][kk], a);
-        acc[i] = a;
-      }
-    }
-  }
-  if (grp == 0) s_ss[j] = ss;
-  __syncthreads();
-  if (j < nr) {
-    const float rstd = rsqrtf(s_ss[j] / (float)hidden + eps);
-#pragma unroll
-    for (int i = 0; i < HEAD_MAXC / 4; ++i) {
-      const int cc = grp * per + i;
-      if (i < per && cc < C) out[(size_t)(rb + j) * C + cc] = rstd * acc[i] + ld_f32<TW>(b + cc);
     }
   }
 }
@@ -418,8 +375,14 @@ static fsdit_status embed_t(float* x, int hidden, int row0, int rows, int kind, 
                (double)rows * hidden * 4.0 * (kind == 0 ? 2.0 : 1.0) + (double)rows * K * 4.0 +
                    (double)hidden * K * sizeof(TW),
                st);
-  embed_kernel<TW><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in, (const TW*)b_in,
-                                           text_proj, (const TW*)mod_emb, temb, modality, time_id, n_times, ea, eb);
+  if (K <= 32)
+    embed_kernel<TW, 32><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
+                                                 (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
+                                                 time_id, n_times, ea, eb);
+  else
+    embed_kernel<TW, 64><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
+                                                 (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
+                                                 time_id, n_times, ea, eb);
   return cuda_check(cudaGetLastError(), "embed_kernel");
 }
 
@@ -455,21 +418,16 @@ fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, in
   return cuda_check(cudaGetLastError(), "time_mlp kernels");
 }
 
-fsdit_status launch_heads(int dtype, const float* x, int row0, int rows, int hidden, const void* g, const void* w,
-                          const void* b, int C, float eps, float* out, cudaStream_t st) {
+fsdit_status launch_rope_table(const int32_t* pos, int rows, int head_dim, int s0, int s1, float log2_theta,
+                               float2* cs, cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
-  const int blocks = (rows + HEAD_ROWS - 1) / HEAD_ROWS;
-  ProfScope ps(PC_HEADS, 1, 2.0 * rows * (double)hidden * C,
-               (double)rows * hidden * 4.0 + (double)C * hidden * (dtype == FSDIT_BF16 ? 2.0 : 4.0) +
-                   (double)rows * C * 4.0,
-               st);
-  if (dtype == FSDIT_BF16)
-    heads_kernel<bf16><<<blocks, 256, 0, st>>>(x, row0, rows, hidden, (const bf16*)g, (const bf16*)w,
-                                               (const bf16*)b, C, eps, out);
-  else
-    heads_kernel<float><<<blocks, 256, 0, st>>>(x, row0, rows, hidden, (const float*)g, (const float*)w,
-                                                (const float*)b, C, eps, out);
-  return cuda_check(cudaGetLastError(), "heads_kernel");
+  const size_t total = (size_t)rows * (head_dim / 2);
+  size_t blocks = (total + 255) / 256;
+  const size_t cap = (size_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  ProfScope ps(PC_ROPE, 1, 0.0, 12.0 * rows + 8.0 * total, st);
+  rope_table_kernel<<<(unsigned)blocks, 256, 0, st>>>(pos, rows, head_dim, s0, s1, log2_theta, cs);
+  return cuda_check(cudaGetLastError(), "rope_table_kernel");
 }
 
 fsdit_status launch_euler(float* x, const float* v, const uint8_t* mod, const uint8_t* mask, int n_rows, int width,

@@ -165,7 +165,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[32];
         tmem_ld32(t_row + (uint32_t)(c * 32), v);
         const int col = nb * BN + c * 32;
-        if (row < args.M && col < args.N) epilogue_row<bf16, 32>(args.ep, row, col, v);
+        if (row < args.M && col < args.N) {
+          if (col + 32 <= args.N) {
+            epilogue_row<bf16, 32>(args.ep, row, col, v);
+          } else {  // ragged last chunk (N % 32 != 0, N even)
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(bar0 + 8 * (2 * STAGES + 2 + buf));
