@@ -131,12 +131,13 @@ def gather_rows(x, pos, keep_idx, n_grid, stream=None):
     return xc, posc
 
 
-def broadcast_residual(x, yc, keep_idx, near_idx, n_grid, out=None, stream=None):
+def broadcast_residual(x, yc, keep_idx, near_idx, grid, out=None, stream=None):
     n_rows, hidden = x.shape
+    T, H, W = grid
     if out is None:
         out = torch.empty_like(x)
     L.call("fsdit_broadcast_residual", L.ptr(x), L.ptr(yc), L.ptr(out), L.ptr(keep_idx),
-           L.ptr(near_idx), keep_idx.numel(), n_grid, n_rows, hidden, _stream(stream))
+           L.ptr(near_idx), keep_idx.numel(), T, H, W, n_rows, hidden, _stream(stream))
     return out
 
 

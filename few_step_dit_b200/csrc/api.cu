@@ -42,8 +42,8 @@ fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* ne
 fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
                            int n_keep, int n_grid, int n_rows, int hidden, cudaStream_t st);
 fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
-                              const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
-                              cudaStream_t st);
+                              const int32_t* near_idx, int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
+                              int hidden, cudaStream_t st);
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
                                  cudaStream_t st);
 fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
@@ -443,22 +443,25 @@ fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, float* x_c, i
 }
 
 fsdit_status fsdit_broadcast_residual(const float* x, const float* y_c, float* out, const int32_t* keep_idx,
-                                      const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
-                                      fsdit_stream_t stream) {
+                                      const int32_t* near_idx, int n_keep, int grid_t, int grid_h, int grid_w,
+                                      int n_rows, int hidden, fsdit_stream_t stream) {
   FS_TRY(need(x, "x"));
   FS_TRY(need(y_c, "y_c"));
   FS_TRY(need(out, "out"));
   FS_TRY(need(keep_idx, "keep_idx"));
   FS_TRY(need(near_idx, "near_idx"));
-  if (n_keep <= 0 || n_grid < n_keep || n_rows < n_grid || hidden <= 0 || hidden % 4 != 0) {
-    set_error("broadcast: need 0 < n_keep <= n_grid <= n_rows and hidden %% 4 == 0");
+  const long long n_grid = (long long)grid_t * grid_h * grid_w;
+  if (grid_t <= 0 || grid_h <= 0 || grid_w <= 0 || n_keep != fsdit_keep_count(grid_t, grid_h, grid_w) ||
+      n_rows < n_grid || hidden <= 0 || hidden % 4 != 0) {
+    set_error("broadcast: need a non-empty grid, n_keep == its kept count, n_rows >= grid rows, hidden %% 4 == 0");
     return FSDIT_E_SHAPE;
   }
   if (out == y_c) {
     set_error("broadcast: out must not alias y_c");
     return FSDIT_E_SHAPE;
   }
-  return launch_broadcast(x, y_c, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, (cudaStream_t)stream);
+  return launch_broadcast(x, y_c, out, keep_idx, near_idx, n_keep, grid_t, grid_h, grid_w, n_rows, hidden,
+                          (cudaStream_t)stream);
 }
 
 fsdit_status fsdit_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
@@ -544,12 +547,8 @@ fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_block_weights
   FS_TRY(launch_gather(x_in, tok->pos_thw, ws.xc, ws.posc, tok->keep_idx, tok->n_keep, n_grid, n, dims->hidden, st));
   FS_TRY(rope_table(dims, ws.posc, n_c, ws.rope, st));
   FS_TRY(block_body(dims, w, ws.xc, ws.xc, ws.posc, ws.rope, n_c, ws, st));
-  if (x_out != x_in) {
-    FS_TRY(launch_broadcast(x_in, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, n, dims->hidden, st));
-  } else {
-    FS_TRY(launch_broadcast(x_out, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, n, dims->hidden,
-                            st));
-  }
+  FS_TRY(launch_broadcast(x_in, ws.xc, x_out, tok->keep_idx, tok->near_idx, tok->n_keep, tok->grid_t, tok->grid_h,
+                          tok->grid_w, n, dims->hidden, st));
   return FSDIT_OK;
 }
 
@@ -624,7 +623,8 @@ static fsdit_status stack_forward_impl(const fsdit_dims* dims, int n_layers, con
       FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, bw.rope_c, n_c, bw, st));
       ++l;
     }
-    FS_TRY(launch_broadcast(x, bw.xc, x, tok->keep_idx, tok->near_idx, tok->n_keep, n_grid, N, H, st));
+    FS_TRY(launch_broadcast(x, bw.xc, x, tok->keep_idx, tok->near_idx, tok->n_keep, tok->grid_t, tok->grid_h,
+                            tok->grid_w, N, H, st));
   }
   // heads: final RMSNorm into the GEMM operand buffer, then the two projections
   FS_TRY(launch_rmsnorm_cast(x, io->g_out, bw.xn, N, H, dims->rms_eps, dims->dtype, st));

@@ -1,11 +1,9 @@
 // HBM-bound kernels of the hot path: keep-index map, gather, nearest-kept
-// broadcast + residual, RMSNorm-cast, embedding, timestep MLP, output heads
-// and the per-modality Euler step.  All rows are moved with 16-byte vector
-// accesses; grids are sized from the SM count.
+// broadcast + residual, RMSNorm-cast, RoPE table, embedding, timestep MLP and
+// the per-modality Euler step.  Rows move with 16-byte vector accesses.
 #include "common.cuh"
 
 namespace fsdit {
-
 
 // ---------------------------------------------------------------- keep map
 
@@ -49,35 +47,43 @@ __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* _
 }
 
 // ---------------------------------------------------------------- broadcast
-// phase 0: every row (out != x); phase 1: dropped grid rows only; phase 2:
-// kept grid rows and non-grid rows (phases 1 then 2 make the in-place form).
-__global__ void broadcast_kernel(const float* __restrict__ x, const float* __restrict__ yc,
-                                 float* __restrict__ out, const int32_t* __restrict__ keep_idx,
-                                 const int32_t* __restrict__ near_idx, int n_keep, int n_grid,
-                                 int n_rows, int hidden, int phase) {
+// Block b < n_keep owns kept token b and every grid row whose nearest kept
+// token it is.  Those rows are its own row src = keep_idx[b] and, because a
+// dropped index takes the kept index just below it on each axis, the rows
+// among src+1, src+W, src+W+1 (same frame) whose near_idx is b.  The block
+// reads y_c[b] and x[src] once: out[src] = y_c[b], out[p] = x[p] + (y_c[b] -
+// x[src]) for the others.  No two blocks touch the same row, so out may equal
+// x.  Blocks b >= n_keep copy the non-grid rows (text, audio, control).
+__global__ void broadcast_kernel(const float* x, const float* __restrict__ yc, float* out,
+                                 const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ near_idx,
+                                 int n_keep, int grid_h, int grid_w, int n_grid, int n_rows, int hidden) {
   const int h4 = hidden >> 2;
-  for (int p = blockIdx.x; p < n_rows; p += gridDim.x) {
-    float4* o = reinterpret_cast<float4*>(out + (size_t)p * hidden);
-    if (p < n_grid) {
-      const int c = near_idx[p];
-      const int src = keep_idx[c];
-      const float4* y = reinterpret_cast<const float4*>(yc + (size_t)c * hidden);
-      if (src == p) {
-        if (phase == 1) continue;
-        for (int i = threadIdx.x; i < h4; i += blockDim.x) o[i] = __ldg(y + i);
-      } else {
-        if (phase == 2) continue;
-        const float4* xp = reinterpret_cast<const float4*>(x + (size_t)p * hidden);
-        const float4* xk = reinterpret_cast<const float4*>(x + (size_t)src * hidden);
-        for (int i = threadIdx.x; i < h4; i += blockDim.x) {
-          const float4 a = xp[i], b = __ldg(y + i), k = xk[i];
-          o[i] = make_float4(a.x + (b.x - k.x), a.y + (b.y - k.y), a.z + (b.z - k.z), a.w + (b.w - k.w));
-        }
-      }
-    } else {
-      if (phase == 1) continue;
-      const float4* y = reinterpret_cast<const float4*>(yc + (size_t)(n_keep + p - n_grid) * hidden);
+  const int n_blocks = n_keep + (n_rows - n_grid);
+  for (int b = blockIdx.x; b < n_blocks; b += gridDim.x) {
+    const float4* y = reinterpret_cast<const float4*>(yc + (size_t)b * hidden);
+    if (b >= n_keep) {
+      float4* o = reinterpret_cast<float4*>(out + (size_t)(n_grid + b - n_keep) * hidden);
       for (int i = threadIdx.x; i < h4; i += blockDim.x) o[i] = __ldg(y + i);
+      continue;
+    }
+    const int src = keep_idx[b];
+    const int w = src % grid_w, h = (src / grid_w) % grid_h;
+    int child[3];
+    int nc = 0;
+    if (w + 1 < grid_w && near_idx[src + 1] == b) child[nc++] = src + 1;
+    if (h + 1 < grid_h && near_idx[src + grid_w] == b) child[nc++] = src + grid_w;
+    if (w + 1 < grid_w && h + 1 < grid_h && near_idx[src + grid_w + 1] == b) child[nc++] = src + grid_w + 1;
+    const float4* xk = reinterpret_cast<const float4*>(x + (size_t)src * hidden);
+    float4* ok = reinterpret_cast<float4*>(out + (size_t)src * hidden);
+    for (int i = threadIdx.x; i < h4; i += blockDim.x) {
+      const float4 yv = __ldg(y + i), kv = xk[i];
+      const float4 d = make_float4(yv.x - kv.x, yv.y - kv.y, yv.z - kv.z, yv.w - kv.w);
+      for (int c = 0; c < nc; ++c) {
+        const float4 a = reinterpret_cast<const float4*>(x + (size_t)child[c] * hidden)[i];
+        reinterpret_cast<float4*>(out + (size_t)child[c] * hidden)[i] =
+            make_float4(a.x + d.x, a.y + d.y, a.z + d.z, a.w + d.w);
+      }
+      ok[i] = yv;
     }
   }
 }
@@ -88,7 +94,6 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
   if (l == 0) red[w] = v;
   __syncthreads();
   float s = 0.f;
@@ -97,14 +102,14 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
-template <typename TO, typename TG>
-__device__ __forceinline__ void store4(TO* o, float a, float b, float c, float d);
+template <typename T>
+__device__ __forceinline__ void store4(T* o, float a, float b, float c, float d);
 template <>
-__device__ __forceinline__ void store4<float, float>(float* o, float a, float b, float c, float d) {
+__device__ __forceinline__ void store4<float>(float* o, float a, float b, float c, float d) {
   *reinterpret_cast<float4*>(o) = make_float4(a, b, c, d);
 }
 template <>
-__device__ __forceinline__ void store4<bf16, bf16>(bf16* o, float a, float b, float c, float d) {
+__device__ __forceinline__ void store4<bf16>(bf16* o, float a, float b, float c, float d) {
   __nv_bfloat162 h0 = __floats2bfloat162_rn(a, b), h1 = __floats2bfloat162_rn(c, d);
   uint2 u;
   u.x = *reinterpret_cast<uint32_t*>(&h0);
@@ -130,31 +135,29 @@ constexpr int RMS_MAXV = 8;
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_cast_kernel(const float* __restrict__ x, const T* __restrict__ g,
                                                            T* __restrict__ xn, int rows, int hidden, float eps) {
-  __shared__ float red[32];
+  __shared__ float red[8];
   const int h4 = hidden >> 2;
-  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-    const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * hidden);
-    float4 v[RMS_MAXV];
-    float ss = 0.f;
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * hidden);
+  float4 v[RMS_MAXV];
+  float ss = 0.f;
 #pragma unroll
-    for (int k = 0; k < RMS_MAXV; ++k) {
-      const int i = threadIdx.x + k * blockDim.x;
-      if (i < h4) {
-        v[k] = xr[i];
-        ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
-      }
+  for (int k = 0; k < RMS_MAXV; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < h4) {
+      v[k] = xr[i];
+      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
     }
-    const float tot = block_sum(ss, red);
-    const float rstd = rsqrtf(tot / (float)hidden + eps);
-    T* o = xn + (size_t)r * hidden;
+  }
+  const float rstd = rsqrtf(block_sum(ss, red) / (float)hidden + eps);
+  T* o = xn + (size_t)r * hidden;
 #pragma unroll
-    for (int k = 0; k < RMS_MAXV; ++k) {
-      const int i = threadIdx.x + k * blockDim.x;
-      if (i < h4) {
-        const float4 gg = load_g4<T>(g + 4 * i);
-        store4<T, T>(o + 4 * i, v[k].x * rstd * gg.x, v[k].y * rstd * gg.y, v[k].z * rstd * gg.z,
-                     v[k].w * rstd * gg.w);
-      }
+  for (int k = 0; k < RMS_MAXV; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < h4) {
+      const float4 gg = load_g4<T>(g + 4 * i);
+      store4<T>(o + 4 * i, v[k].x * rstd * gg.x, v[k].y * rstd * gg.y, v[k].z * rstd * gg.z, v[k].w * rstd * gg.w);
     }
   }
 }
@@ -178,11 +181,11 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int rows, int
 // ---------------------------------------------------------------- embedding
 // x[r] = src(r) + mod_emb[modality[r]] + temb[time_id[r]], where src(r) is the
 // small-K projection lat[r'] W^T + b of a video/control or audio row, or the
-// precomputed text projection row.  A block owns EMB_ROWS consecutive rows of
-// one segment; each thread keeps one W row in registers and reuses it across
-// the block's rows.
-constexpr int EMB_ROWS = 16;
-constexpr int EMB_MAXK = 64;
+// precomputed text projection row.  A block owns EMB_RB rows of one segment
+// and EMB_CB consecutive columns: each thread keeps its column's weight row
+// in registers; the rows' latents, modality and timestep embeddings of the
+// block's columns are staged in shared memory; stores are coalesced.
+constexpr int EMB_RB = 32, EMB_CB = 256, EMB_MAXT = 8;
 
 template <typename TW, int KMAX>
 __global__ void __launch_bounds__(256) embed_kernel(
@@ -191,49 +194,58 @@ __global__ void __launch_bounds__(256) embed_kernel(
     const float* __restrict__ text_proj, const TW* __restrict__ mod_emb, const float* __restrict__ temb,
     const uint8_t* __restrict__ modality, const uint8_t* __restrict__ time_id, int n_times,
     int expect_a, int expect_b) {
-  __shared__ float s_lat[EMB_ROWS][EMB_MAXK];
-  __shared__ int s_mod[EMB_ROWS], s_tid[EMB_ROWS];
-  const int rb0 = blockIdx.x * EMB_ROWS;
-  const int nr = min(EMB_ROWS, rows - rb0);
-  if (nr <= 0) return;
-  if (threadIdx.x < nr) {
-    const int r = row0 + rb0 + threadIdx.x;
-    int m = modality[r], t = time_id[r];
-    if ((m != expect_a && m != expect_b) || t >= n_times) {
-      raise_device_error(DEVERR_TAGS);
-      m = expect_a;
-      t = 0;
+  __shared__ float s_lat[EMB_RB][KMAX];
+  __shared__ float s_mod[4][EMB_CB];
+  __shared__ float s_temb[EMB_MAXT][EMB_CB];
+  __shared__ int s_m[EMB_RB], s_t[EMB_RB];
+  const int rb0 = blockIdx.x * EMB_RB;
+  const int nr = min(EMB_RB, rows - rb0);
+  const int c = blockIdx.y * EMB_CB + threadIdx.x;
+  const bool col_ok = c < hidden;
+  if (threadIdx.x < EMB_RB) {
+    int m = expect_a, t = 0;
+    if (threadIdx.x < nr) {
+      const int r = row0 + rb0 + threadIdx.x;
+      m = modality[r];
+      t = time_id[r];
+      if ((m != expect_a && m != expect_b) || t >= n_times) {
+        raise_device_error(DEVERR_TAGS);
+        m = expect_a;
+        t = 0;
+      }
     }
-    s_mod[threadIdx.x] = m;
-    s_tid[threadIdx.x] = t;
+    s_m[threadIdx.x] = m;
+    s_t[threadIdx.x] = t;
   }
   if (kind == 1) {
-    for (int i = threadIdx.x; i < EMB_ROWS * KMAX; i += blockDim.x) {
+    for (int i = threadIdx.x; i < EMB_RB * KMAX; i += blockDim.x) {
       const int rr = i / KMAX, kk = i % KMAX;
       s_lat[rr][kk] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
     }
   }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) s_mod[m][threadIdx.x] = col_ok ? ld_f32<TW>(mod_emb + (size_t)m * hidden + c) : 0.f;
+  for (int t = 0; t < n_times; ++t) s_temb[t][threadIdx.x] = col_ok ? temb[(size_t)t * hidden + c] : 0.f;
   __syncthreads();
-  for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
-    float wr[KMAX];  // one weight row in registers (KMAX is a compile-time bound on K)
-    float bias = 0.f;
+  if (!col_ok) return;
+  float wr[KMAX];
+  float bias = 0.f;
+  if (kind == 1) {
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) wr[k] = k < K ? ld_f32<TW>(w_in + (size_t)c * K + k) : 0.f;
+    bias = ld_f32<TW>(b_in + c);
+  }
+  for (int j = 0; j < nr; ++j) {
+    float acc;
     if (kind == 1) {
+      acc = bias;
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k) wr[k] = k < K ? ld_f32<TW>(w_in + (size_t)c * K + k) : 0.f;
-      bias = ld_f32<TW>(b_in + c);
+      for (int k = 0; k < KMAX; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
+    } else {
+      acc = text_proj[(size_t)(rb0 + j) * hidden + c];
     }
-    for (int j = 0; j < nr; ++j) {
-      float acc;
-      if (kind == 1) {
-        acc = bias;
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
-      } else {
-        acc = text_proj[(size_t)(rb0 + j) * hidden + c];
-      }
-      acc += ld_f32<TW>(mod_emb + (size_t)s_mod[j] * hidden + c) + temb[(size_t)s_tid[j] * hidden + c];
-      x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
-    }
+    acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
+    x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
   }
 }
 
@@ -242,9 +254,8 @@ __global__ void __launch_bounds__(256) embed_kernel(
 // sinusoidal features of 1000*t computed in shared memory.
 struct Times8 { float t[8]; };
 template <typename TW>
-__global__ void time_mlp1_kernel(Times8 times, int n_times, int t_freq,
-                                 const TW* __restrict__ w1, const TW* __restrict__ b1,
-                                 float* __restrict__ h1, int hidden) {
+__global__ void time_mlp1_kernel(Times8 times, int n_times, int t_freq, const TW* __restrict__ w1,
+                                 const TW* __restrict__ b1, float* __restrict__ h1, int hidden) {
   extern __shared__ float s_feat[];  // [n_times][t_freq]
   const int half = t_freq / 2;
   for (int i = threadIdx.x; i < n_times * half; i += blockDim.x) {
@@ -273,8 +284,28 @@ __global__ void time_mlp1_kernel(Times8 times, int n_times, int t_freq,
   }
 }
 
-// Stage 2: temb[t, c] = sum_k h1[t,k] W2[c,k] + b2[c]; W2 read once.
+// Stage 2: temb[t, c] = sum_k h1[t,k] W2[c,k] + b2[c]; one warp per output
+// column, 8 weights (16 bytes of bf16) per lane per step, W2 read once.
 constexpr int TMLP_MAXT = 8;
+template <typename TW>
+__device__ __forceinline__ void load8(const TW* p, float* w);
+template <>
+__device__ __forceinline__ void load8<bf16>(const bf16* p, float* w) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t a[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a[i]));
+    w[2 * i] = f.x;
+    w[2 * i + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* w) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
+
 template <typename TW>
 __global__ void time_mlp2_kernel(const float* __restrict__ h1, int n_times, const TW* __restrict__ w2,
                                  const TW* __restrict__ b2, float* __restrict__ temb, int hidden) {
@@ -284,11 +315,18 @@ __global__ void time_mlp2_kernel(const float* __restrict__ h1, int n_times, cons
     float acc[TMLP_MAXT];
 #pragma unroll
     for (int t = 0; t < TMLP_MAXT; ++t) acc[t] = 0.f;
-    for (int k = lane; k < hidden; k += 32) {
-      const float wv = ld_f32<TW>(w2 + (size_t)c * hidden + k);
+    for (int k = lane * 8; k < hidden; k += 256) {
+      float w[8];
+      load8<TW>(w2 + (size_t)c * hidden + k, w);
 #pragma unroll
-      for (int t = 0; t < TMLP_MAXT; ++t)
-        if (t < n_times) acc[t] = fmaf(h1[(size_t)t * hidden + k], wv, acc[t]);
+      for (int t = 0; t < TMLP_MAXT; ++t) {
+        if (t < n_times) {
+          const float4 ha = __ldg(reinterpret_cast<const float4*>(h1 + (size_t)t * hidden + k));
+          const float4 hb = __ldg(reinterpret_cast<const float4*>(h1 + (size_t)t * hidden + k) + 1);
+          acc[t] += ha.x * w[0] + ha.y * w[1] + ha.z * w[2] + ha.w * w[3] + hb.x * w[4] + hb.y * w[5] + hb.z * w[6] +
+                    hb.w * w[7];
+        }
+      }
     }
 #pragma unroll
     for (int t = 0; t < TMLP_MAXT; ++t) {
@@ -336,31 +374,26 @@ fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_
 }
 
 fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
-                              const int32_t* near_idx, int n_keep, int n_grid, int n_rows, int hidden,
-                              cudaStream_t st) {
-  const int g = grid_for_rows(n_rows, 8);
-  const double n_c = (double)n_keep + (n_rows - n_grid);
-  ProfScope ps(PC_BCAST, out != x ? 1 : 2, 0.0, ((double)n_grid + n_c + n_rows) * hidden * 4.0, st);
-  if (out != x) {
-    broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 0);
-    return cuda_check(cudaGetLastError(), "broadcast_kernel");
-  }
-  broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 1);
-  fsdit_status s = cuda_check(cudaGetLastError(), "broadcast_kernel(dropped rows)");
-  if (s != FSDIT_OK) return s;
-  broadcast_kernel<<<g, 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, n_grid, n_rows, hidden, 2);
-  return cuda_check(cudaGetLastError(), "broadcast_kernel(kept rows)");
+                              const int32_t* near_idx, int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
+                              int hidden, cudaStream_t st) {
+  const int n_grid = grid_t * grid_h * grid_w;
+  const int n_blocks = n_keep + (n_rows - n_grid);
+  // unique bytes: every grid row of x read once, y_c read once, every row written once
+  ProfScope ps(PC_BCAST, 1, 0.0, ((double)n_grid + n_blocks + n_rows) * hidden * 4.0, st);
+  broadcast_kernel<<<grid_for_rows(n_blocks, 8), 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, grid_h,
+                                                               grid_w, n_grid, n_rows, hidden);
+  return cuda_check(cudaGetLastError(), "broadcast_kernel");
 }
 
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
                                  cudaStream_t st) {
-  const int grid = grid_for_rows(rows, 8);
+  if (rows <= 0) return FSDIT_OK;
   const double s = dtype == FSDIT_BF16 ? 2.0 : 4.0;
   ProfScope ps(PC_NORM, 1, 0.0, (double)rows * hidden * (4.0 + s) + hidden * s, st);
   if (dtype == FSDIT_BF16)
-    rmsnorm_cast_kernel<bf16><<<grid, 256, 0, st>>>(x, (const bf16*)g, (bf16*)xn, rows, hidden, eps);
+    rmsnorm_cast_kernel<bf16><<<rows, 256, 0, st>>>(x, (const bf16*)g, (bf16*)xn, rows, hidden, eps);
   else
-    rmsnorm_cast_kernel<float><<<grid, 256, 0, st>>>(x, (const float*)g, (float*)xn, rows, hidden, eps);
+    rmsnorm_cast_kernel<float><<<rows, 256, 0, st>>>(x, (const float*)g, (float*)xn, rows, hidden, eps);
   return cuda_check(cudaGetLastError(), "rmsnorm_cast_kernel");
 }
 
@@ -370,19 +403,19 @@ static fsdit_status embed_t(float* x, int hidden, int row0, int rows, int kind, 
                             const float* temb, const uint8_t* modality, const uint8_t* time_id, int n_times,
                             int ea, int eb, cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
-  const int blocks = (rows + EMB_ROWS - 1) / EMB_ROWS;
+  dim3 grid((rows + EMB_RB - 1) / EMB_RB, (hidden + EMB_CB - 1) / EMB_CB);
   ProfScope ps(PC_EMBED, 1, 2.0 * rows * (double)hidden * K,
                (double)rows * hidden * 4.0 * (kind == 0 ? 2.0 : 1.0) + (double)rows * K * 4.0 +
                    (double)hidden * K * sizeof(TW),
                st);
   if (K <= 32)
-    embed_kernel<TW, 32><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
-                                                 (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
-                                                 time_id, n_times, ea, eb);
+    embed_kernel<TW, 32><<<grid, EMB_CB, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
+                                                  (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
+                                                  time_id, n_times, ea, eb);
   else
-    embed_kernel<TW, 64><<<blocks, 256, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
-                                                 (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
-                                                 time_id, n_times, ea, eb);
+    embed_kernel<TW, 64><<<grid, EMB_CB, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
+                                                  (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
+                                                  time_id, n_times, ea, eb);
   return cuda_check(cudaGetLastError(), "embed_kernel");
 }
 
@@ -400,20 +433,21 @@ fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, i
 fsdit_status launch_time_mlp(int dtype, const float* times_host, int n_times, int t_freq, const void* w1,
                              const void* b1, const void* w2, const void* b2, float* h1, float* temb, int hidden,
                              cudaStream_t st) {
-  const int blocks = num_sms() * 2;
   const size_t sm1 = (size_t)n_times * t_freq * sizeof(float);
   ProfScope ps(PC_TIMEMLP, 2, 2.0 * n_times * (double)hidden * (t_freq + hidden),
                (double)hidden * (t_freq + hidden) * (dtype == FSDIT_BF16 ? 2.0 : 4.0), st);
   Times8 times_dev;
   for (int i = 0; i < 8; ++i) times_dev.t[i] = i < n_times ? times_host[i] : 0.f;
+  const int blocks1 = num_sms() * 2;
+  const int blocks2 = (hidden + 7) / 8;  // one warp per output column
   if (dtype == FSDIT_BF16) {
-    time_mlp1_kernel<bf16><<<blocks, 256, sm1, st>>>(times_dev, n_times, t_freq, (const bf16*)w1, (const bf16*)b1,
-                                                     h1, hidden);
-    time_mlp2_kernel<bf16><<<blocks, 256, 0, st>>>(h1, n_times, (const bf16*)w2, (const bf16*)b2, temb, hidden);
+    time_mlp1_kernel<bf16><<<blocks1, 256, sm1, st>>>(times_dev, n_times, t_freq, (const bf16*)w1, (const bf16*)b1,
+                                                      h1, hidden);
+    time_mlp2_kernel<bf16><<<blocks2, 256, 0, st>>>(h1, n_times, (const bf16*)w2, (const bf16*)b2, temb, hidden);
   } else {
-    time_mlp1_kernel<float><<<blocks, 256, sm1, st>>>(times_dev, n_times, t_freq, (const float*)w1,
-                                                      (const float*)b1, h1, hidden);
-    time_mlp2_kernel<float><<<blocks, 256, 0, st>>>(h1, n_times, (const float*)w2, (const float*)b2, temb, hidden);
+    time_mlp1_kernel<float><<<blocks1, 256, sm1, st>>>(times_dev, n_times, t_freq, (const float*)w1,
+                                                       (const float*)b1, h1, hidden);
+    time_mlp2_kernel<float><<<blocks2, 256, 0, st>>>(h1, n_times, (const float*)w2, (const float*)b2, temb, hidden);
   }
   return cuda_check(cudaGetLastError(), "time_mlp kernels");
 }

@@ -85,9 +85,33 @@ def case_block(a):
     return res
 
 
+def case_memory(a):
+    """Full-width gather, broadcast (in place) and RMSNorm-cast on a grid."""
+    w = S.WORKLOADS[a.workload]
+    T, H, W = w.grid
+    n = w.n_tokens
+    g = torch.Generator(device="cuda").manual_seed(3)
+    x = torch.randn(n, w.hidden, generator=g, device="cuda")
+    pos = torch.zeros(n, 3, dtype=torch.int32, device="cuda")
+    keep_idx, near_idx = api.keep_map(T, H, W)
+    n_keep = keep_idx.numel()
+    xc, posc = api.gather_rows(x, pos, keep_idx, w.n_video)
+    gain = torch.ones(w.hidden, dtype=torch.bfloat16, device="cuda")
+    res = {"case": "memory", "workload": a.workload, "rows": n, "kept": n_keep}
+    hb = w.hidden * 4.0
+    ms = time_it(lambda: api.gather_rows(x, pos, keep_idx, w.n_video), a.iters, a.warmup)
+    res["gather_ms"], res["gather_gbs"] = ms, xc.shape[0] * hb * 2 / ms / 1e6
+    ms = time_it(lambda: api.broadcast_residual(x, xc, keep_idx, near_idx, w.grid, out=x), a.iters, a.warmup)
+    res["broadcast_ms"] = ms
+    res["broadcast_gbs"] = (w.n_video + xc.shape[0] + n) * hb / ms / 1e6
+    ms = time_it(lambda: api.rmsnorm_cast(x, gain), a.iters, a.warmup)
+    res["rmsnorm_ms"], res["rmsnorm_gbs"] = ms, n * w.hidden * 6.0 / ms / 1e6
+    return res
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("case", choices=["attention", "gemm", "block"])
+    p.add_argument("case", choices=["attention", "gemm", "block", "memory"])
     p.add_argument("--n", type=int, default=12560)
     p.add_argument("--heads", type=int, default=56)
     p.add_argument("--M", type=int, default=12560)
@@ -100,7 +124,8 @@ def main():
     a = p.parse_args()
     B.build()
     L.load()
-    res = {"attention": case_attention, "gemm": case_gemm, "block": case_block}[a.case](a)
+    res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
+           "memory": case_memory}[a.case](a)
     api.device_error()
     print(json.dumps(res), flush=True)
 

@@ -77,7 +77,7 @@ _SIGS = {
                                                 C.POINTER(Tokens), _I]),
     "fsdit_build_keep_map": (_I, [_I, _I, _I, _P, _P, _P]),
     "fsdit_gather_rows": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
-    "fsdit_broadcast_residual": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "fsdit_broadcast_residual": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "fsdit_rmsnorm_cast": (_I, [_P, _P, _P, _I, _I, _F, _I, _P]),
     "fsdit_linear": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "fsdit_attention": (_I, [C.POINTER(Dims), _P, _P, _I, _P]),

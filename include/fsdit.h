@@ -193,11 +193,14 @@ FSDIT_API fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, flo
  * section): the compressed layers' update of kept token c is
  * d_c = y_c[c] - x[keep_idx[c]]; kept grid rows take y_c, dropped grid rows p
  * take x[p] + d_{near_idx[p]} (float32 arithmetic), non-grid rows take their
- * y_c rows.  out may equal x (then it runs in two ordered launches). */
+ * y_c rows.  The grid is grid_t x grid_h x grid_w (rows [0, T*H*W) of x) with
+ * the map of fsdit_build_keep_map (n_keep kept tokens); each kept token's
+ * dropped rows lie at +1 / +W / +W+1 of it in its frame.  One launch; out may
+ * equal x (every row is read and written by one block only). */
 FSDIT_API fsdit_status fsdit_broadcast_residual(const float* x, const float* y_c, float* out,
                                       const int32_t* keep_idx, const int32_t* near_idx,
-                                      int n_keep, int n_grid, int n_rows, int hidden,
-                                      fsdit_stream_t stream);
+                                      int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
+                                      int hidden, fsdit_stream_t stream);
 
 /* RMSNorm fused into the GEMM-operand pass: xn[r] = cast(x[r] * g /
  * sqrt(mean(x[r]^2) + eps)).  x float32 [rows, hidden]; g and xn in `dtype`. */

@@ -68,7 +68,8 @@ def test_entry_points_reject_null_and_bad_shapes_without_launching(fs):
     assert fs.fsdit_linear(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 64, 2, s) == -1
     assert fs.fsdit_build_keep_map(0, 9, 10, fake, fake, s) == -2
     assert fs.fsdit_gather_rows(fake, None, fake, None, fake, 0, 10, 10, 64, s) == -2
-    assert fs.fsdit_broadcast_residual(fake, fake, fake, fake, fake, 5, 4, 10, 64, s) == -2
+    assert fs.fsdit_broadcast_residual(fake, fake, fake, fake, fake, 5, 1, 3, 3, 10, 64, s) == -2  # 4 kept
+    assert fs.fsdit_broadcast_residual(fake, fake, fake, fake, fake, 4, 1, 3, 3, 8, 64, s) == -2   # rows < grid
     assert fs.fsdit_rmsnorm_cast(fake, fake, fake, 4, 100, 1e-6, 1, s) == -2
     assert fs.fsdit_rmsnorm_cast(fake, fake, fake, 4, 64, 1e-6, 3, s) == -4
     tc = (C.c_float * 4)(0, 0.2, 0.5, 0)

@@ -81,7 +81,7 @@ def test_broadcast_residual(grid, n_other, hidden, in_place):
     ref = O.broadcast_residual(x.numpy(), yc.numpy(), keep_idx, near_idx, V)
     k_dev, n_dev = api.keep_map(T, H, W)
     xd = x.to(DEV)
-    out = api.broadcast_residual(xd, yc.to(DEV), k_dev, n_dev, V, out=xd if in_place else None)
+    out = api.broadcast_residual(xd, yc.to(DEV), k_dev, n_dev, grid, out=xd if in_place else None)
     torch.cuda.synchronize()
     got = out.cpu().numpy()
     kept = np.zeros(V, bool)
