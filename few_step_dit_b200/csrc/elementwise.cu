@@ -185,7 +185,7 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int rows, int
 // and EMB_CB consecutive columns: each thread keeps its column's weight row
 // in registers; the rows' latents, modality and timestep embeddings of the
 // block's columns are staged in shared memory; stores are coalesced.
-constexpr int EMB_RB = 32, EMB_CB = 256, EMB_MAXT = 8;
+constexpr int EMB_RB = 128, EMB_CB = 256, EMB_MAXT = 8;
 
 template <typename TW, int KMAX>
 __global__ void __launch_bounds__(256) embed_kernel(

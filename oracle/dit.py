@@ -213,6 +213,39 @@ def dit_block(x, w, pos, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
     return h + linear(u, w["w_2"], w["b_2"])
 
 
+def dit_block_rows(x, w, pos, heads, head_dim, rows, rope_split=(32, 48, 48), eps=1e-6,
+                   theta=10000.0):
+    """``dit_block(x, ...)[rows]`` computed for the requested rows only.
+
+    Keys and values are formed for every row (each output row attends to all
+    of them); queries, the output projection and the FFN only for ``rows``.
+    Same definition as ``dit_block``, restricted -- used to check outputs of
+    full-size blocks one row at a time."""
+    x = np.asarray(x, dtype=F64)
+    n = x.shape[0]
+    rows = np.asarray(rows, dtype=np.int64)
+    A = heads * head_dim
+    xn = rms_norm(x, w["g_attn"], eps)
+    w_qkv = np.asarray(w["w_qkv"], dtype=F64)
+    b_qkv = np.asarray(w["b_qkv"], dtype=F64)
+    q = linear(xn[rows], w_qkv[:A], b_qkv[:A]).reshape(len(rows), heads, head_dim)
+    k = linear(xn, w_qkv[A:2 * A], b_qkv[A:2 * A]).reshape(n, heads, head_dim)
+    v = linear(xn, w_qkv[2 * A:], b_qkv[2 * A:]).reshape(n, heads, head_dim)
+    q = apply_rope(q, np.asarray(pos)[rows], rope_split, theta)
+    k = apply_rope(k, pos, rope_split, theta)
+    scale = 1.0 / math.sqrt(head_dim)
+    a = np.empty((len(rows), heads, head_dim), dtype=F64)
+    for h in range(heads):
+        s = (q[:, h, :] @ k[:, h, :].T) * scale
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        a[:, h, :] = p @ v[:, h, :]
+    hrow = x[rows] + linear(a.reshape(len(rows), A), w["w_o"], w["b_o"])
+    u = gelu_tanh(linear(rms_norm(hrow, w["g_ffn"], eps), w["w_1"], w["b_1"]))
+    return hrow + linear(u, w["w_2"], w["b_2"])
+
+
 # ---------------------------------------------------------------------------
 # Compressed block: gather kept rows, run the block, broadcast back.
 # ---------------------------------------------------------------------------
@@ -264,6 +297,25 @@ def dit_block_compressed(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video
     pos_c = gather_rows(pos, keep_idx, n_video)
     y_c = dit_block(x_c, w, pos_c, heads, head_dim, rope_split, eps, theta)
     return broadcast_residual(x, y_c, keep_idx, near_idx, n_video)
+
+
+def dit_block_compressed_rows(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video, rows,
+                              rope_split=(32, 48, 48), eps=1e-6, theta=10000.0):
+    """``dit_block_compressed(...)[rows]`` for the requested rows only: the
+    compressed block is evaluated (via ``dit_block_rows``) just for the
+    compressed rows those outputs read, then the same broadcast rule applies."""
+    x = np.asarray(x, dtype=F64)
+    rows = np.asarray(rows, dtype=np.int64)
+    keep_idx = np.asarray(keep_idx, dtype=np.int64)
+    near_idx = np.asarray(near_idx, dtype=np.int64)
+    n_keep = keep_idx.shape[0]
+    need = np.unique(np.where(rows < n_video, near_idx[np.minimum(rows, n_video - 1)],
+                              n_keep + rows - n_video))
+    x_c = gather_rows(x, keep_idx, n_video)
+    pos_c = gather_rows(pos, keep_idx, n_video)
+    y_c = np.zeros_like(x_c)
+    y_c[need] = dit_block_rows(x_c, w, pos_c, heads, head_dim, need, rope_split, eps, theta)
+    return broadcast_residual(x, y_c, keep_idx, near_idx, n_video)[rows]
 
 
 # ---------------------------------------------------------------------------

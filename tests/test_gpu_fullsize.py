@@ -1,0 +1,139 @@
+"""Full-size parity: the full-width Flash block on the 6x34x60 grid (12,560
+tokens, hidden 5376, 56 heads, FFN 14336, bf16) in the launch configuration the
+bench uses, checked on sampled output rows that the oracle computes one by one
+(relative L2 <= 1e-2 on the rows and on their update y - x); plus the
+standard model's control-frame packing through the stack and the 4-evaluation
+sampler at small width."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from few_step_dit_b200 import api, build, lib as L
+from few_step_dit_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    L.load()
+    yield
+    torch.cuda.synchronize()
+    api.device_error()
+
+
+@pytest.fixture(scope="module")
+def full_block():
+    w = S.WORKLOADS["flash_block_6x34x60"]
+    layers, _ = S.make_weights(w, n_layers=1)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    return w, layers[0], inp["x"].float(), tags
+
+
+def _sample_rows(w, seed=11):
+    V, N = w.n_video, w.n_tokens
+    T, H, W = w.grid
+    fixed = [0, 1, W, W + 1, W - 1, (H - 1) * W, H * W - 1, H * W, V - 1, V - 2, V - W,
+             V, V + 1, V + w.n_text - 1, N - w.n_audio, N - 1]
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([fixed, rng.integers(0, N, 32)]))
+
+
+@pytest.mark.parametrize("compress", [True, False])
+def test_full_width_block_sampled_rows(full_block, compress):
+    w, wts, x, tags = full_block
+    dims = api.dims_of(w)
+    seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
+    bw = api.BlockWeights({k: v.to(DEV) for k, v in wts.items()})
+    y = api.block_forward(dims, bw, seq, x.to(DEV), compress=compress)
+    torch.cuda.synchronize()
+    rows = _sample_rows(w)
+    got = y[torch.as_tensor(rows, device=DEV)].double().cpu().numpy()
+    wn = S.to_numpy64(wts)
+    xn = x.double().numpy()
+    if compress:
+        k, n = O.keep_map(*w.grid)
+        ref = O.dit_block_compressed_rows(xn, wn, tags["pos"], w.heads, w.head_dim, k, n, w.n_video, rows)
+    else:
+        ref = O.dit_block_rows(xn, wn, tags["pos"], w.heads, w.head_dim, rows)
+    assert O.rel_l2(got, ref) < 1e-2
+    assert O.rel_l2(got - xn[rows], ref - xn[rows]) < 1e-2
+
+
+def test_full_width_block_properties_at_every_row(full_block):
+    # properties that hold at any size: kept and non-grid rows of the
+    # compressed block equal the block on the gathered sequence; every dropped
+    # row's update equals its nearest kept row's update (fp32 rounding only)
+    w, wts, x, tags = full_block
+    dims = api.dims_of(w)
+    seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
+    bw = api.BlockWeights({k: v.to(DEV) for k, v in wts.items()})
+    xd = x.to(DEV)
+    y = api.block_forward(dims, bw, seq, xd, compress=True)
+    xc, posc = api.gather_rows(xd, seq.pos, seq.keep_idx, w.n_video)
+    # the same block on the gathered rows, no compression, same kernels
+    tags_c = {k: v for k, v in tags.items()}
+    keep = seq.keep_idx.long()
+    sel = torch.cat([keep, torch.arange(w.n_video, w.n_tokens, device=DEV)])
+    tags_c["pos"] = seq.pos[sel].cpu().numpy()
+    seq_c = api.Sequence(tags_c | {"modality": tags["modality"][:sel.numel()],
+                                   "time_id": tags["time_id"][:sel.numel()],
+                                   "out_mask": tags["out_mask"][:sel.numel()]},
+                         (0, 0, 0), seq.n_keep, w.n_text, w.n_audio, DEV, compress=False)
+    yc = api.block_forward(dims, bw, seq_c, xc, compress=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y[sel], yc)
+    src = keep[seq.near_idx.long()]
+    d = (y[:w.n_video] - xd[:w.n_video]) - (y[src] - xd[src])
+    scale = (y[:w.n_video] - xd[:w.n_video]).abs().max()
+    assert float(d.abs().max()) <= 1e-5 * float(scale) + 1e-5
+
+
+def test_stack_with_control_frames_matches_oracle():
+    # standard-model packing: target grid + clean control frames whose RoPE
+    # time is 16 below the target's, at small width, fp32
+    w = S.scaled(S.WORKLOADS["tiny_block_f32"], control_frames=1, n_layers=3, compress=(0, 0, 0),
+                 video_clock=(1.0, 0.2), audio_clock=(1.0, 0.5))
+    layers, io = S.make_weights(w)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    assert (tags["modality"] == 3).sum() == w.n_control
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vv, va = bb.forward(seq, [0.0, 1.0, 1.0], inp["video_lat"].to(DEV), inp["text_emb"].to(DEV),
+                        inp["audio_lat"].to(DEV))
+    torch.cuda.synchronize()
+    rv, ra = O.dit_stack([S.to_numpy64(l) for l in layers], w.compress, S.to_numpy64(io), tags,
+                         [0.0, 1.0, 1.0], inp["video_lat"].double().numpy(), inp["text_emb"].double().numpy(),
+                         inp["audio_lat"].double().numpy(), w.heads, w.head_dim)
+    assert O.rel_l2(vv.double().cpu().numpy(), rv) < 1e-5
+    assert O.rel_l2(va.double().cpu().numpy(), ra) < 1e-5
+
+
+def test_standard_four_eval_sampler_moves_only_target_rows():
+    w = S.scaled(S.WORKLOADS["standard_backbone_12x34x60"], hidden=256, heads=2, ffn=512, grid=(2, 5, 6),
+                 control_frames=1, n_text=16, n_audio=8, n_layers=2, compress=(0, 0), dtype="f32")
+    layers, io = S.make_weights(w)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vl, al = inp["video_lat"].to(DEV).clone(), inp["audio_lat"].to(DEV).clone()
+    bb.sample(seq, w.video_clock, w.audio_clock, vl, inp["text_emb"].to(DEV), al)
+    torch.cuda.synchronize()
+    rv, ra = O.flow_sample([S.to_numpy64(l) for l in layers], w.compress, S.to_numpy64(io), tags,
+                           w.video_clock, w.audio_clock, inp["video_lat"].double().numpy(),
+                           inp["text_emb"].double().numpy(), inp["audio_lat"].double().numpy(), w.heads,
+                           w.head_dim)
+    got = vl.double().cpu().numpy()
+    assert O.rel_l2(got, rv) < 1e-5 and O.rel_l2(al.double().cpu().numpy(), ra) < 1e-5
+    # control rows are clean conditions: untouched by all 4 Euler steps
+    ctrl = slice(w.n_video, w.n_video + w.n_control)
+    assert np.array_equal(got[ctrl], inp["video_lat"].double().numpy()[ctrl])

@@ -374,6 +374,21 @@ def test_broadcast_dropped_rows_carry_nearest_kept_update():
     assert np.abs(y[dropped] - y[src[dropped]]).min() > 0
 
 
+def test_row_restricted_block_equals_full_block_rows():
+    rng = np.random.default_rng(24)
+    T, Hg, Wg = 2, 5, 6
+    x, pos, V, w = _grid_case(rng, T, Hg, Wg, 5)
+    rows = np.array([0, 3, 7, 13, V - 1, V, x.shape[0] - 1])
+    full = O.dit_block(x, w, pos, 2, 128)
+    np.testing.assert_allclose(O.dit_block_rows(x, w, pos, 2, 128, rows), full[rows], rtol=1e-12,
+                               atol=1e-12)
+    keep_idx, near_idx = O.keep_map(T, Hg, Wg)
+    comp = O.dit_block_compressed(x, w, pos, 2, 128, keep_idx, near_idx, V)
+    np.testing.assert_allclose(
+        O.dit_block_compressed_rows(x, w, pos, 2, 128, keep_idx, near_idx, V, rows), comp[rows],
+        rtol=1e-12, atol=1e-12)
+
+
 def test_segment_form_equals_per_layer_form():
     rng = np.random.default_rng(23)
     T, Hg, Wg = 2, 5, 6
