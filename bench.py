@@ -16,7 +16,7 @@ the fp64 CPU oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
-import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -30,13 +30,16 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from few_step_dit_b200 import api, build as B, lib as L  # noqa: E402
+from few_step_dit_b200 import api, build as B, lib as L, replicas as R  # noqa: E402
 from few_step_dit_b200 import synthetic as S  # noqa: E402
 
 METRIC = "Flash backbone ms/3-eval pass and tokens/s on 1 B200; % of bf16 tensor peak"
 UNIT = "tokens/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["few_step_dit_b200/csrc/gemm_tc.cu", "few_step_dit_b200/csrc/common.cuh",
+                "few_step_dit_b200/csrc/tc_ptx.cuh"]
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "gemm_traffic_flash_backbone_6x34x60.json")
 
 
 def parse():
@@ -49,16 +52,37 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-full-compare", action="store_true",
                    help="skip timing the same backbone with compression off")
+    p.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     return p.parse_args()
 
 
 def load_peaks():
     try:
         with open(PEAKS_PATH) as f:
-            d = json.load(f)
-        return d, "measured"
+            return json.load(f), "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_sources_sha256():
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic(workload):
+    """DRAM bytes per GEMM launch from the committed ncu capture of this
+    workload, or None when there is none or the GEMM sources changed since."""
+    try:
+        with open(TRAFFIC_PATH) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("workload") != workload or d.get("sources_sha256") != gemm_sources_sha256():
+        return None
+    return d.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------- clocks
@@ -109,56 +133,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ---------------------------------------------------------------- CPU oracle sample
-
-def oracle_sample(w, reps=1):
-    """Time the fp64 oracle on one token-compressed full-width block of the
-    workload (its kept video rows + text + audio) and project a full pass.
-
-    Returns (tokens_per_s, seconds_per_pass, sample_description, threads)."""
-    import numpy as np
-
-    import oracle as O
-
-    T, H, W = w.grid
-    k, _ = O.keep_map(T, H, W)
-    n_c = len(k) + w.n_tokens - w.n_video
-    g = torch.Generator().manual_seed(S.SEED_WEIGHTS)
-    wts = S.to_numpy64(S.make_block_weights(w, g))
-    rng = np.random.default_rng(S.SEED_INPUTS)
-    x = rng.standard_normal((n_c, w.hidden))
-    tags = S.pack_tokens(w)
-    pos = O.gather_rows(tags["pos"], k, w.n_video)
-    times = []
-    for _ in range(reps):
-        t0 = time.perf_counter()
-        O.dit_block(x, wts, pos, w.heads, w.head_dim)
-        times.append(time.perf_counter() - t0)
-    t_c = statistics.median(times)
-    # a full-resolution layer scales by its algorithmic FLOPs
-    f_c = block_flops(w, n_c)
-    f_f = block_flops(w, w.n_tokens)
-    t_f = t_c * f_f / f_c
-    n_comp = sum(1 for c in w.compress if c)
-    n_full = len(w.compress) - n_comp
-    per_pass = w.n_evals * (n_comp * t_c + n_full * t_f)
-    threads = blas_threads()
-    desc = (f"one token-compressed full-width block ({n_c} rows, hidden {w.hidden}) timed in fp64 "
-            f"numpy ({t_c:.2f} s); full layers scaled by FLOPs ({f_f / f_c:.2f}x); pass = "
-            f"{w.n_evals} evals x ({n_comp} compressed + {n_full} full layers)")
-    return w.n_tokens * w.n_evals / per_pass, per_pass, desc, threads
-
-
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:  # noqa: BLE001
-        pass
-    return len(os.sched_getaffinity(0))
-
+# ---------------------------------------------------------------- work counts
 
 def block_flops(w, n):
     """Algorithmic FLOPs of one block on n rows: qkv, output, two FFN
@@ -177,9 +152,60 @@ def pass_flops(w, compressed=True):
     return tot * w.n_evals
 
 
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(w, reps=1):
+    """Time the fp64 oracle on one token-compressed full-width block of the
+    workload (its kept video rows + text + audio; the full sequence when the
+    workload has no compressed layer) and project a full pass by FLOPs.
+
+    Returns (tokens_per_s, seconds_per_pass, sample_description, threads)."""
+    import numpy as np
+
+    import oracle as O
+
+    T, H, W = w.grid
+    comp = any(w.compress)
+    k, _ = O.keep_map(T, H, W)
+    n_s = len(k) + w.n_tokens - w.n_video if comp else w.n_tokens
+    g = torch.Generator().manual_seed(S.SEED_WEIGHTS)
+    wts = S.to_numpy64(S.make_block_weights(w, g))
+    rng = np.random.default_rng(S.SEED_INPUTS)
+    x = rng.standard_normal((n_s, w.hidden))
+    tags = S.pack_tokens(w)
+    pos = O.gather_rows(tags["pos"], k, w.n_video) if comp else tags["pos"]
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        O.dit_block(x, wts, pos, w.heads, w.head_dim)
+        times.append(time.perf_counter() - t0)
+    t_s = statistics.median(times)
+    f_s = block_flops(w, n_s)
+    n_comp = sum(1 for c in w.compress if c)
+    per_pass = 0.0
+    for c in w.compress:
+        per_pass += t_s * block_flops(w, n_s if c else w.n_tokens) / f_s
+    per_pass *= w.n_evals
+    desc = (f"one {'token-compressed ' if comp else ''}full-width block ({n_s} rows, hidden {w.hidden}) "
+            f"timed in fp64 numpy ({t_s:.2f} s); other layers scaled by FLOPs; pass = {w.n_evals} evals x "
+            f"({n_comp} compressed + {len(w.compress) - n_comp} full layers)")
+    return w.n_tokens * w.n_evals / per_pass, per_pass, desc, blas_threads()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return len(os.sched_getaffinity(0))
+
+
 # ---------------------------------------------------------------- reference arm
 
-def run_reference(args, rank, world):
+def run_reference(args, rank):
     if rank != 0:
         return
     w = S.WORKLOADS[args.workload]
@@ -214,7 +240,7 @@ def build_backbone(w, device, rank):
     tags = S.pack_tokens(w)
     seq = api.Sequence.from_workload(w, tags, device)
     bb = api.Backbone(dims, bw, iow, w.compress)
-    inp = S.make_inputs(w, device="cpu", seed=S.SEED_INPUTS + rank)
+    inp = S.make_inputs(w, device="cpu", seed=R.input_seed(S.SEED_INPUTS, rank))
     return bb, seq, inp
 
 
@@ -229,23 +255,6 @@ def timed(fn, steps, stream):
     return start.elapsed_time(end)
 
 
-def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def barrier(world):
-    torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-
-
 def run_fsdit(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -253,7 +262,6 @@ def run_fsdit(args, rank, world, local_rank):
     L.load()
     w = S.WORKLOADS[args.workload]
     bb, seq, inp = build_backbone(w, device, rank)
-    stream = torch.cuda.current_stream()
     vl0 = inp["video_lat"].to(device)
     al0 = inp["audio_lat"].to(device)
     text = inp["text_emb"].to(device)
@@ -268,18 +276,39 @@ def run_fsdit(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     api.device_error()
-    barrier(world)
+    R.barrier(world, device)
+
+    # capture one pass in a CUDA graph; the library's event profiler is active
+    # during the capture, so its event pairs replay with every launch
+    L.profile_start(20000)
+    graph, launch_mode = None, "eager"
+    if not args.eager:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step()
+            graph, launch_mode = g, "cuda_graph"
+        except Exception as e:  # noqa: BLE001
+            launch_mode = f"eager (graph capture failed: {type(e).__name__})"
+            torch.cuda.synchronize()
+            L.profile_stop()
+            L.profile_start(20000)
+    run = graph.replay if graph is not None else step
+    if graph is not None:
+        run()  # one untimed replay
+    stream = torch.cuda.current_stream()
     clocks = ClockSampler(local_rank)
-    L.profile_start(200000)
-    barrier(world)
-    t_ms = timed(step, args.steps, stream)
-    barrier(world)
-    prof = L.profile_stop()
+    R.barrier(world, device)
+    t_ms = timed(run, args.steps, stream)
+    R.barrier(world, device)
     clk = clocks.stop()
+    prof = L.profile_stop()  # the last pass's launches (graph) / all passes (eager)
+    prof_steps = 1 if graph is not None else args.steps
     api.device_error()
-    t_ms = max_over_ranks(t_ms, world)
+    t_ms = R.max_over_ranks(t_ms, world, device)
     ms_per_step = t_ms / args.steps
-    value = world * w.n_tokens * w.n_evals / (ms_per_step / 1000.0)
+    value = R.weak_scaling_value(w.n_tokens * w.n_evals, world, ms_per_step / 1000.0)
+    del graph
 
     # end to end through the public API: pinned host inputs -> device, sample, result -> host
     pin = {k: v.pin_memory() for k, v in inp.items() if k in ("video_lat", "audio_lat", "text_emb")}
@@ -295,18 +324,18 @@ def run_fsdit(args, rank, world, local_rank):
         out_a.copy_(al, non_blocking=True)
 
     e2e_step()
-    barrier(world)
-    e_ms = max_over_ranks(timed(e2e_step, args.steps, stream), world) / args.steps
+    R.barrier(world, device)
+    e_ms = R.max_over_ranks(timed(e2e_step, args.steps, stream), world, device) / args.steps
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = out_v.numel() * 4 + out_a.numel() * 4
 
     # same backbone with compression off (the pages' ablation)
     full_ms = None
-    if not args.no_full_compare:
+    if not args.no_full_compare and any(w.compress):
         step(compress=False)
-        barrier(world)
+        R.barrier(world, device)
         n_full = max(1, min(args.steps, 2))
-        full_ms = max_over_ranks(timed(lambda: step(False), n_full, stream), world) / n_full
+        full_ms = R.max_over_ranks(timed(lambda: step(False), n_full, stream), world, device) / n_full
 
     peaks, peak_src = load_peaks()
     gemm = {k: v for k, v in prof.items() if k.startswith("gemm")}
@@ -317,14 +346,13 @@ def run_fsdit(args, rank, world, local_rank):
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     kernels = {}
     for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"]):
-        e = {"launches": v["launches"], "ms_per_step": v["ms"] / args.steps}
+        e = {"launches_per_step": v["launches"] // prof_steps, "ms_per_step": v["ms"] / prof_steps}
         if v["flops"] > 0 and k.startswith(("gemm", "attention")):
             e["tflops"] = v["flops"] / (v["ms"] / 1e3) / 1e12
         if v["bytes"] > 0 and not k.startswith(("gemm", "attention")):
             e["gbs"] = v["bytes"] / (v["ms"] / 1e3) / 1e9
         kernels[k] = e
-    launches = sum(v["launches"] for v in prof.values())
-    tot_flops = pass_flops(w)
+    launches_per_step = sum(v["launches"] for v in prof.values()) // prof_steps
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -332,16 +360,19 @@ def run_fsdit(args, rank, world, local_rank):
         "config": {"workload": args.workload, "layers": w.n_layers, "evals": w.n_evals,
                    "grid": "x".join(map(str, w.grid)), "tokens": w.n_tokens,
                    "kept_video_tokens": seq.n_keep, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: the 22.7 GB of bf16 weights stream from HBM every eval"},
-        "tensor_peak_frac": (tot_flops / (ms_per_step / 1e3) / 1e12) / peak,
+                   "launch": launch_mode,
+                   "l2": "inputs larger than L2: the bf16 weights (22.7 GB for 42 layers) stream from HBM "
+                         "every evaluation"},
+        "tensor_peak_frac": (pass_flops(w) / (ms_per_step / 1e3) / 1e12) / peak,
         "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel (all projections)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak if peak else None, "traffic": None,
+                     "frac": achieved / peak if peak else None,
+                     "traffic": gemm_traffic(args.workload),
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "launches_per_step": g_n / args.steps},
+                     "launches_per_step": g_n // prof_steps},
         "kernels": kernels,
-        "gpu_launches": launches,
-        "e2e": {"value": world * w.n_tokens * w.n_evals / (e_ms / 1000.0), "unit": UNIT,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": R.weak_scaling_value(w.n_tokens * w.n_evals, world, e_ms / 1000.0), "unit": UNIT,
                 "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
     if full_ms is not None:
@@ -359,22 +390,17 @@ def run_fsdit(args, rank, world, local_rank):
 
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = R.env()
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        run_reference(args, rank)
         return
     if world > 1:
-        import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    R.init(world, backend="nccl")
     try:
         run_fsdit(args, rank, world, local_rank)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        R.shutdown(world)
 
 
 if __name__ == "__main__":

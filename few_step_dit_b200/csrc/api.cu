@@ -25,6 +25,16 @@ struct Prof {
 };
 static Prof g_prof;
 
+// Inside a stream capture the event pair must be recorded as external event
+// nodes, so every replay of the graph stamps them.
+static void prof_record(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, st);
+}
+
 ProfScope::ProfScope(int c, int k, double fl, double by, cudaStream_t s) : slot(-1), st(s) {
   if (!g_prof.on || 2 * (size_t)(g_prof.used + 1) > g_prof.ev.size()) return;
   slot = g_prof.used++;
@@ -32,10 +42,10 @@ ProfScope::ProfScope(int c, int k, double fl, double by, cudaStream_t s) : slot(
   g_prof.kernels[slot] = k;
   g_prof.flops[slot] = fl;
   g_prof.bytes[slot] = by;
-  cudaEventRecord(g_prof.ev[2 * slot], st);
+  prof_record(g_prof.ev[2 * slot], st);
 }
 ProfScope::~ProfScope() {
-  if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
+  if (slot >= 0) prof_record(g_prof.ev[2 * slot + 1], st);
 }
 
 fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st);

@@ -158,6 +158,38 @@ def test_bf16_stack_small_width():
     assert O.rel_l2(ga, ra) < 1e-2
 
 
+def test_sampler_cuda_graph_replay_equals_eager():
+    # the whole few-step pass is launch-only host code, so it captures into one
+    # CUDA graph; a replay must reproduce the eager result bit for bit
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=4, compress=(0, 1, 1, 0))
+    layers, io, inp, tags = _setup(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vl0, al0, text = inp["video_lat"].to(DEV), inp["audio_lat"].to(DEV), inp["text_emb"].to(DEV)
+    vl, al = vl0.clone(), al0.clone()
+
+    def step():
+        vl.copy_(vl0)
+        al.copy_(al0)
+        bb.sample(seq, w.video_clock, w.audio_clock, vl, text, al)
+
+    step()
+    torch.cuda.synchronize()
+    ref_v, ref_a = vl.clone(), al.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    vl.zero_()
+    al.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(vl, ref_v) and torch.equal(al, ref_a)
+    del g
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_sampler_matches_oracle(dtype):
     w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512,
