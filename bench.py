@@ -364,7 +364,7 @@ def run_fsdit(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: the bf16 weights (22.7 GB for 42 layers) stream from HBM "
                          "every evaluation"},
         "tensor_peak_frac": (pass_flops(w) / (ms_per_step / 1e3) / 1e12) / peak,
-        "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel (all projections)",
+        "roofline": {"bound": "tensor", "kernel": "tc_gemm_pair_kernel (all projections with M > 128)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak if peak else None,
                      "traffic": gemm_traffic(args.workload),

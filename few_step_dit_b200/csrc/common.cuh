@@ -147,6 +147,109 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
   }
 }
 
+// ------------------------------------------------ tensor-core GEMM epilogue
+// The bf16 tensor-core kernels hold one accumulator row per thread in chunks
+// of 32 columns.  Everything a chunk needs besides its accumulators (bias, the
+// RoPE (cos, sin) pairs or the fp32 residual) is loaded by epi32_prefetch
+// before the accumulators are read out of TMEM, so the two latencies overlap.
+struct Epi32Pre {
+  uint4 bias[4];    // 32 bf16 bias values (the same for every row)
+  float4 extra[8];  // QKV_ROPE: 16 (cos, sin) pairs; RESIDUAL: 32 fp32 residual values
+};
+
+// GELU (tanh form) with the hardware tanh approximation (relative error about
+// 2^-11), used where the result is rounded to bf16 (2^-9) next.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float gelu_tanh_bf16out(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  const float k1 = 0.044715f;
+  return 0.5f * x * (1.0f + tanh_approx(k0 * (x + k1 * x * x * x)));
+}
+
+// Columns [col, col + 32) of `row`, all inside the output (col + 32 <= N);
+// bias, out, resid and rope_cs 16-byte aligned, head_dim a power of two.
+__device__ __forceinline__ void epi32_prefetch(const EpiParams& p, int row, int col, Epi32Pre& e) {
+  const uint4* b = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(p.bias) + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) e.bias[i] = __ldg(b + i);
+  if (p.epi == FSDIT_EPI_QKV_ROPE) {
+    if (col < p.rope_cols && p.rope_cs != nullptr) {
+      const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (size_t)row * (p.head_dim >> 1) +
+                                                         ((col & (p.head_dim - 1)) >> 1));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e.extra[i] = __ldg(cs + i);
+    }
+  } else if (p.epi == FSDIT_EPI_RESIDUAL) {
+    const float4* r = reinterpret_cast<const float4*>(p.resid + (size_t)row * p.ldr + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e.extra[i] = r[i];
+  }
+}
+
+__device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col, float* v, const Epi32Pre& e) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&e.bias[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * i + 2 * j] += f.x;
+      v[8 * i + 2 * j + 1] += f.y;
+    }
+  }
+  if (p.epi == FSDIT_EPI_QKV_ROPE) {
+    if (col < p.rope_cols && p.rope_cs == nullptr) {
+      const int32_t* pos3 = p.pos + (size_t)row * 3;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2)
+        rope_pair(v[i], v[i + 1], (col + i) & (p.head_dim - 1), p.s0, p.s1, p.head_dim, pos3, p.log2_theta);
+    } else if (col < p.rope_cols) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 t = e.extra[i];  // (cos, sin) of pairs 2i and 2i+1
+        float a = v[4 * i], b = v[4 * i + 1];
+        v[4 * i] = a * t.x - b * t.y;
+        v[4 * i + 1] = a * t.y + b * t.x;
+        a = v[4 * i + 2];
+        b = v[4 * i + 3];
+        v[4 * i + 2] = a * t.z - b * t.w;
+        v[4 * i + 3] = a * t.w + b * t.z;
+      }
+    }
+  } else if (p.epi == FSDIT_EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_bf16out(v[i]);
+  }
+  if (p.epi == FSDIT_EPI_RESIDUAL) {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 r = e.extra[i];
+      o[i] = make_float4(r.x + v[4 * i], r.y + v[4 * i + 1], r.z + v[4 * i + 2], r.w + v[4 * i + 3]);
+    }
+  } else if (p.epi == FSDIT_EPI_BIAS_F32) {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+        u[j] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      o[i] = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  }
+}
+
 }  // namespace fsdit
 
 // Host-side internal API shared by the .cu files.

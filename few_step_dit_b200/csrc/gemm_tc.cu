@@ -189,6 +189,202 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace gemm
 
+// Pair-tile variant: a cluster of two CTAs computes a 256 x 256 output tile
+// with tcgen05.mma.cta_group::2.  Each CTA stages only its own 128 A rows and
+// 128 of the 256 B rows per K step (32 KB a stage instead of 48 KB for the
+// same 128 x 256 share of the output), which halves the B operand's
+// shared-memory and L2 traffic per FLOP.  Roles per CTA as above; warp 1 of
+// CTA rank 0 issues the pair MMAs.  Both CTAs' TMA copies of a stage complete
+// on rank 0's `full` barrier (rank 0 expects the bytes of both); the MMA
+// commits release the stage in both CTAs.  Accumulator rows 0..127 of a tile
+// sit in rank 0's TMEM, 128..255 in rank 1's; each CTA's epilogue stores its
+// own rows and releases the accumulator buffer on rank 0's barrier (one arrive
+// per warp).
+namespace gemm2 {
+
+constexpr int BM = 256, BN = 256, BK = 64;
+constexpr int HM = BM / 2, HN = BN / 2;  // per-CTA share of A rows and B rows
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HM * BK * 2;
+constexpr int B_BYTES = HN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each on half the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+// barrier ids: full[s] = s (rank 0's counts both CTAs' copies), empty[s] = S+s,
+// tfull[b] = 2S+b, tempty[b] = 2S+2+b (rank 0 only), drain = 2S+4
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
+constexpr int GROUP_N = 8;
+constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, 0);
+
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const gemm::Args args) {
+  using namespace ptx;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  auto FULL = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+  auto EMPTY = [&](int s) { return bar0 + 8u * (uint32_t)(STAGES + s); };
+  auto TFULL = [&](int b) { return bar0 + 8u * (uint32_t)(2 * STAGES + b); };
+  auto TEMPTY = [&](int b) { return bar0 + 8u * (uint32_t)(2 * STAGES + 2 + b); };
+  const uint32_t DRAIN = bar0 + 8u * (uint32_t)(2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + STAGES * STAGE_BYTES + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(FULL(s), 1);
+      mbar_init(EMPTY(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(TFULL(b), 1);
+      mbar_init(TEMPTY(b), 2 * EPI_WARPS);  // epilogue warps of both CTAs
+    }
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int num_tiles = args.tiles_m * args.tiles_n;
+  const int KB = (args.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int last_s = -1;
+      uint32_t last_ph = 0;
+      bool ok = true;
+      const uint32_t full0 = peer_addr(FULL(0), 0u);  // rank 0's full barriers
+      for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
+        int mb, nb;
+        gemm::tile_coords(tile, args, mb, nb);
+        const int row_a = mb * BM + (int)rank * HM, row_b = nb * BN + (int)rank * HN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(EMPTY(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t full = full0 + 8u * (uint32_t)s;
+          if (rank == 0) mbar_expect_tx(FULL(s), 2 * STAGE_BYTES);
+          tma_load_2d_pair(sa, &tmA, kb * BK, row_a, full);
+          tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, row_b, full);
+          last_s = s;
+          last_ph = ph;
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      // on abort, let the newest copies land before the CTA can exit (rank 1
+      // cannot observe rank 0's barrier; its copies finish within microseconds)
+      if (!ok && last_s >= 0) {
+        if (rank == 0) mbar_wait(FULL(last_s), last_ph, nullptr);
+        else spin_cycles(1LL << 22);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // pair MMA issuer
+      const uint32_t empty_peer0 = peer_addr(EMPTY(0), 1u), tfull_peer0 = peer_addr(TFULL(0), 1u);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++it) {
+        const int buf = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait_cluster(TEMPTY(buf), aph ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(FULL(s), ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + s * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC,
+                             (kb | k) != 0 ? 1u : 0u);
+          tc_commit_pair(EMPTY(s));
+          tc_commit_pair(empty_peer0 + 8u * (uint32_t)s);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(TFULL(buf));
+        tc_commit_pair(tfull_peer0 + 8u * (uint32_t)buf);
+      }
+      // every MMA this thread issued has completed (and stopped reading both
+      // CTAs' shared memory) once `drain` flips
+      tc_commit_pair(DRAIN);
+      mbar_wait(DRAIN, 0, nullptr);
+    }
+  } else {
+    const int q = warp & 3;                    // TMEM lane quarter this warp may access
+    const int c0 = ((warp - 2) >> 2) * (BN / 64);  // first of its BN/64 column chunks
+    const uint32_t tempty0 = peer_addr(TEMPTY(0), 0u);
+    int it = 0;
+    for (int tile = cid; tile < num_tiles; tile += ncl, ++it) {
+      const int buf = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      int mb, nb;
+      gemm::tile_coords(tile, args, mb, nb);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(TFULL(buf), aph, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = mb * BM + (int)rank * HM + q * 32 + lane;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      const bool row_ok = row < args.M;
+#pragma unroll 1
+      for (int c = c0; c < c0 + BN / 64; ++c) {
+        const int col = nb * BN + c * 32;
+        const bool full = row_ok && col + 32 <= args.N;
+        Epi32Pre pre;
+        if (full) epi32_prefetch(args.ep, row, col, pre);
+        float v[32];
+        tmem_ld32(t_row + (uint32_t)(c * 32), v);
+        if (full) {
+          epi32_apply(args.ep, row, col, v, pre);
+        } else if (row_ok && col < args.N) {  // ragged last chunk (N % 32 != 0, N even)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(TEMPTY(buf));
+        else mbar_arrive_cluster(tempty0 + 8u * (uint32_t)buf);
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm2
+
 // ---------------------------------------------------------------- host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
@@ -222,8 +418,83 @@ fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uin
   return FSDIT_OK;
 }
 
+// How many CTA pairs of tc_gemm_pair_kernel fit on the device at once
+// (0: the pair kernel cannot run, use the single-CTA kernel).
+static int pair_clusters_resident() {
+  static std::once_flag once;
+  static int n = 0;
+  std::call_once(once, [] {
+    if (cudaFuncSetAttribute(gemm2::tc_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm2::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm2::tc_gemm_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
+            cudaSuccess) {
+      (void)cudaGetLastError();
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(gemm2::THREADS);
+    cfg.dynamicSmemBytes = gemm2::SMEM_BYTES;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel, &cfg) == cudaSuccess) n = c;
+    (void)cudaGetLastError();
+  });
+  return n;
+}
+
+static fsdit_status launch_linear_pair(const void* a, const void* w, const EpiParams& ep, int M, int N, int K,
+                                       int clusters, cudaStream_t st) {
+  using namespace gemm2;
+  CUtensorMap tmA, tmB;
+  fsdit_status s = make_tmap_bf16(&tmA, a, (uint64_t)M, (uint64_t)K, (uint64_t)K, HM, BK);
+  if (s != FSDIT_OK) return s;
+  s = make_tmap_bf16(&tmB, w, (uint64_t)N, (uint64_t)K, (uint64_t)K, HN, BK);
+  if (s != FSDIT_OK) return s;
+  gemm::Args args;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.tiles_m = (M + BM - 1) / BM;
+  args.tiles_n = (N + BN - 1) / BN;
+  args.group_n = GROUP_N < args.tiles_n ? GROUP_N : args.tiles_n;
+  args.ep = ep;
+  const int tiles = args.tiles_m * args.tiles_n;
+  const int ncl = tiles < clusters ? tiles : clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * ncl);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel, tmA, tmB, args), "tc_gemm_pair_kernel");
+}
+
 fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep, int M, int N, int K,
                               cudaStream_t st) {
+  // pair tiles once there are two 128-row blocks to share them; their
+  // epilogue moves bias, output, residual and RoPE table in 16-byte pieces
+  auto a16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  const bool f32_out = ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32;
+  const bool vec_ok = a16(ep.bias) && a16(ep.out) && ep.ldo % (f32_out ? 4 : 8) == 0 &&
+                      (ep.epi != FSDIT_EPI_RESIDUAL || (a16(ep.resid) && ep.ldr % 4 == 0)) &&
+                      (ep.rope_cs == nullptr || a16(ep.rope_cs)) && (ep.head_dim & (ep.head_dim - 1)) == 0;
+  if (M > gemm2::HM && vec_ok) {
+    const int clusters = pair_clusters_resident();
+    if (clusters > 0) return launch_linear_pair(a, w, ep, M, N, K, clusters, st);
+  }
   using namespace gemm;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;

@@ -136,6 +136,12 @@ LIN_CASES = [
     (200, 512, 256, L.EPI_GELU),
     (200, 256, 512, L.EPI_RESIDUAL),
     (77, 256, 520, L.EPI_BIAS_F32),
+    # 256 x 256 pair tiles: the second column tile's upper half (cols 384..511)
+    # lies wholly past N, K = 136 ends in a partial 64-wide step
+    (513, 352, 136, L.EPI_BIAS),
+    # 11 x 8 = 88 pair tiles, more than the CTA pairs resident on a B200, so
+    # pairs run several tiles and reuse both accumulator buffers
+    (2600, 2048, 256, L.EPI_GELU),
     (3668, 5376, 5376, L.EPI_RESIDUAL),
 ]
 
