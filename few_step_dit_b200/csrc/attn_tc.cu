@@ -54,6 +54,77 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max of 128 values as eight independent chains of three-input max (depth 8
+// plus a 3-level combine) instead of one 127-long dependent chain.
+__device__ __forceinline__ float row_max128(const float* s) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float a = max3(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+    for (int i = 3; i < 15; i += 2) a = max3(a, s[k + 8 * i], s[k + 8 * (i + 1)]);
+    mx[k] = fmaxf(a, s[k + 8 * 15]);
+  }
+  return max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
+// ---- packed fp32 pairs (f32x2 FMA-pipe instructions of sm_100) ----
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float a, float b) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(f2_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+  f2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
+  f2_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b) {
+  f2_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair on the FMA pipe, x <= 0: x = j + f with j = round(x) (the
+// 1.5 * 2^23 shifter leaves j in the low mantissa bits) and f in [-1/2, 1/2];
+// 2^f from a cubic fitted to 2^f on that interval (relative error below
+// 7.5e-5, far under the bf16 rounding P gets next); j is added to the exponent
+// field as an integer.  Inputs below -125 are clamped (their 2^x underflows
+// bf16 P anyway).
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  const f2_t x = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const f2_t shifter = f2(12582912.0f, 12582912.0f);
+  const f2_t t = f2_add(x, shifter);
+  const f2_t fr = f2_sub(x, f2_sub(t, shifter));
+  f2_t q = f2_fma(f2(0.0551716577f, 0.0551716577f), fr, f2(0.242611121f, 0.242611121f));
+  q = f2_fma(q, fr, f2(0.693260988f, 0.693260988f));
+  q = f2_fma(q, fr, f2(0.999928074f, 0.999928074f));
+  float t0, t1, q0, q1;
+  f2_split(t, t0, t1);
+  f2_split(q, q0, q1);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// One pair in EMU_EVERY is exponentiated on the FMA pipe (0: none), taking
+// that share of the work off the MUFU pipe.
+constexpr int EMU_EVERY = 0;
+
 // O (+)= P V with P [128 x 16k] in TMEM (A operand) and V in shared memory.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -97,7 +168,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(B_KEMPTY + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
       mbar_init(bar(B_SFULL + s), 1);   // per query tile
-      mbar_init(bar(B_PFULL + s), 128); // per query tile
+      mbar_init(bar(B_PFULL + s), 4);   // per query tile: one arrive per softmax warp
       mbar_init(bar(B_ODONE + s), 1);   // per query tile
     }
     mbar_init(bar(B_DRAIN), 1);
@@ -215,18 +286,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!w_ok) { ok = false; break; }
       tc_fence_after();
       float s[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) tmem_ld32(tmem + lane_addr + s_col + (uint32_t)(c * 32), s + c * 32);
+      tmem_ld128(tmem + lane_addr + s_col, s);
       const int valid = n - j * BKV;  // keys past n are masked
       if (valid < BKV) {
 #pragma unroll
         for (int c = 0; c < BKV; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
+      const float m_cand = row_max128(s) * sl2;
       const bool grow = m_cand > m + RESCALE_THRESHOLD;
       const float m_new = grow ? m_cand : m;
       const float corr = grow ? ex2(m - m_new) : 1.0f;
@@ -243,23 +310,31 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(ta, u);
         }
       }
-      float sum = 0.f;
+      const f2_t scale2 = f2(sl2, sl2), negm2 = f2(-m_new, -m_new);
+      f2_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // four independent partial row sums (pairs)
+      uint32_t pk[BKV / 2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2(fmaf(s[h * 64 + c], sl2, -m_new));
-          const float p1 = ex2(fmaf(s[h * 64 + c + 1], sl2, -m_new));
-          sum += p0 + p1;
-          pk[c >> 1] = pack_bf16(p0, p1);
+      for (int c = 0; c < BKV; c += 2) {
+        float x0, x1, p0, p1;
+        f2_split(f2_fma(f2(s[c], s[c + 1]), scale2, negm2), x0, x1);
+        if (EMU_EVERY > 0 && (c >> 1) % EMU_EVERY == EMU_EVERY - 1) {
+          exp2_poly_pair(x0, x1, p0, p1);
+        } else {
+          p0 = ex2(x0);
+          p1 = ex2(x1);
         }
-        tmem_st32(tmem + lane_addr + s_col + (uint32_t)(h * 32), pk);
+        acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2(p0, p1));
+        pk[c >> 1] = pack_bf16(p0, p1);
       }
+      tmem_st64(tmem + lane_addr + s_col, pk);
+      float a0, a1;
+      f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+      const float sum = a0 + a1;
       l = l * corr + sum;
       m = m_new;
       tc_fence_before();
-      mbar_arrive(bar(B_PFULL + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PFULL + t));
     }
     if (ok && nkv > 0) {
       int w_ok = 1;
@@ -295,6 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 }  // namespace attn
+
 
 fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int attn_w, cudaStream_t st) {
   using namespace attn;
