@@ -14,13 +14,21 @@ Sources (web write-ups of arXiv 2609.15863, "LynnReal-Omni"):
   layer schedule and spatial token compression).
 * [PaperDaily] longzhangge PaperDaily, "LynnReal Lab视频恢复与生成：统一多模态控制，
   Flash降至377毫秒", section 一 (input tags, control offset, dual clocks) and
-  section 二 "Flash怎么把22帧压到377毫秒" (compression, residual broadcast).
+  section 二 "Flash怎么把22帧压到377毫秒" (compression, residual broadcast),
+  section 三 "长视频不是无限塞历史，而是保留“够用的记忆”" (chunked long video).
+* [tokendh] section "长视频生成：怎么记住十分钟前发生的事" (boundary frame,
+  bounded multi-stride history).
+
+Modules: ``dit.py`` (block, compression, stack, flow-matching sampler) and
+``long_video.py`` (chunked generation with the bounded history; import it as
+``oracle.long_video``).
 
 Every floating-point step runs in float64.  Where the pages leave a step open
 the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
 
 Parity status per function: everything in ``dit.py`` is pinned by the CPU
-tests in ``tests/test_oracle_pins.py`` except the conventions that are pure
+tests in ``tests/test_oracle_pins.py`` and everything in ``long_video.py`` by
+``tests/test_oracle_long_video.py``, except the conventions that are pure
 definitions (weight init, time-embedding MLP, bias placement); those are
 "parity unpinned" in the sense that no page fixes them, so the GPU path is
 compared against this oracle's definition of them.
