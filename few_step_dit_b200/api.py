@@ -255,3 +255,108 @@ class Backbone:
                C.byref(self.io.struct), C.byref(tok), E, tv, ta, L.ptr(video_lat), L.ptr(text_emb),
                L.ptr(audio_lat), L.ptr(ws), ws.numel(), _stream(stream))
         return video_lat, audio_lat
+
+
+# ---------------------------------------------------------------- long video
+
+class HistoryStore:
+    """Device store of a video's latent frames for the bounded multi-stride
+    history (fsdit_history_*): frame 0 plus the newest capacity-1 frames."""
+
+    def __init__(self, H, W, C_ch, capacity=L.HISTORY_MIN_SLOTS, device="cuda"):
+        lib = L.load()
+        nbytes = lib.fsdit_history_bytes(capacity, H, W, C_ch)
+        self.frames = torch.empty(max(nbytes // 4, 1), dtype=torch.float32, device=device)
+        self.s = L.HistoryStore()
+        self.H, self.W, self.C = H, W, C_ch
+        L.call("fsdit_history_init", C.byref(self.s), L.ptr(self.frames), capacity, H, W, C_ch)
+
+    @property
+    def n_frames(self):
+        return self.s.n_frames
+
+    def push(self, frames, stream=None):
+        """Append latent frames (contiguous fp32, H*W*C values per frame)."""
+        fe = self.H * self.W * self.C
+        assert frames.dtype == torch.float32 and frames.is_contiguous() and frames.numel() % fe == 0
+        L.call("fsdit_history_push", C.byref(self.s), L.ptr(frames), frames.numel() // fe, _stream(stream))
+
+    def plan(self, n_before):
+        """History plan of a chunk whose boundary is frame n_before."""
+        out = (L.HistoryEntry * L.HISTORY_MAX_ENTRIES)()
+        n = L.load().fsdit_history_plan(int(n_before), out, L.HISTORY_MAX_ENTRIES)
+        if n < 0:
+            raise L.FsditError("fsdit_history_plan", n, "bad n_before")
+        return out, n
+
+    def rows(self, plan, n):
+        return L.load().fsdit_history_rows(plan, n, self.H, self.W)
+
+    def gather(self, plan, n, lat, pos, stream=None):
+        """Write the plan's rows into lat [rows, >= C] fp32 and pos [rows, 3] int32."""
+        L.call("fsdit_history_gather", C.byref(self.s), plan, n, L.ptr(lat), lat.stride(0), L.ptr(pos),
+               _stream(stream))
+
+    def copy_frame(self, frame, dst, stream=None):
+        L.call("fsdit_history_copy_frame", C.byref(self.s), int(frame), L.ptr(dst), _stream(stream))
+
+
+def chunk_tags(grid, base, has_boundary, n_hist, n_text, n_audio):
+    """Host row tags of one chunk (fsdit_chunk_tags); history pos rows are left
+    zero for the gather to fill."""
+    T, H, W = grid
+    n = T * H * W + n_hist + n_text + n_audio
+    mod = np.zeros(n, np.uint8)
+    tid = np.zeros(n, np.uint8)
+    out = np.zeros(n, np.uint8)
+    pos = np.zeros((n, 3), np.int32)
+    L.call("fsdit_chunk_tags", T, H, W, int(base), int(bool(has_boundary)), n_hist, n_text, n_audio,
+           mod.ctypes.data, tid.ctypes.data, out.ctypes.data, pos.ctypes.data)
+    return dict(modality=mod, time_id=tid, out_mask=out, pos=pos)
+
+
+class LongVideo:
+    """Chunked long-video generation: each chunk samples [boundary + future
+    latents | history | text | audio] with the few-step sampler and appends its
+    new latent frames to the history store."""
+
+    def __init__(self, backbone: Backbone, grid, n_text, n_audio, video_ch, capacity=L.HISTORY_MIN_SLOTS,
+                 device="cuda"):
+        self.bb = backbone
+        self.grid = tuple(grid)
+        self.n_text, self.n_audio = n_text, n_audio
+        T, H, W = self.grid
+        self.store = HistoryStore(H, W, video_ch, capacity, device)
+        self.device = torch.device(device)
+        self.compress = any(int(c) for c in backbone.compress)
+
+    def prepare(self, stream=None):
+        """Sequence and latent buffer of the next chunk, history gathered, the
+        boundary latent in place.  Returns (seq, video_lat, has_boundary)."""
+        T, H, W = self.grid
+        hw, n_grid = H * W, T * H * W
+        has_b = self.store.n_frames > 0
+        base = self.store.n_frames - 1 if has_b else 0
+        plan, n_plan = self.store.plan(base if has_b else 0)
+        n_hist = self.store.rows(plan, n_plan)
+        tags = chunk_tags(self.grid, base, has_b, n_hist, self.n_text, self.n_audio)
+        seq = Sequence(tags, self.grid, n_grid + n_hist, self.n_text, self.n_audio, self.device,
+                       self.compress, stream)
+        vl = torch.empty(n_grid + n_hist, self.store.C, dtype=torch.float32, device=self.device)
+        if n_hist:
+            self.store.gather(plan, n_plan, vl[n_grid:], seq.pos[n_grid:n_grid + n_hist], stream)
+        return seq, vl, has_b, base
+
+    def chunk(self, noise_video, text_emb, noise_audio, video_clock, audio_clock, stream=None):
+        """Generate one chunk from its initial target latents [T*H*W, C] and
+        audio latents; returns (target latents [T*H*W, C], audio latents)."""
+        T, H, W = self.grid
+        hw, n_grid = H * W, T * H * W
+        seq, vl, has_b, base = self.prepare(stream)
+        vl[:n_grid].copy_(noise_video)
+        if has_b:
+            self.store.copy_frame(base, vl[:hw], stream)
+        al = noise_audio.clone()
+        self.bb.sample(seq, video_clock, audio_clock, vl, text_emb, al, stream=stream)
+        self.store.push(vl[hw:n_grid] if has_b else vl[:n_grid], stream)
+        return vl[:n_grid], al

@@ -15,7 +15,7 @@ namespace fsdit {
 static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "gemm_gelu", "gemm_bias_f32",
                                            "gemm_bias",     "attention",     "rmsnorm_cast", "gather",
                                            "broadcast",     "embed",         "time_mlp",  "heads",
-                                           "euler",         "keep_map",  "rope_table"};
+                                           "euler",         "keep_map",  "rope_table", "history_gather"};
 struct Prof {
   bool on = false;
   int used = 0;

@@ -259,7 +259,7 @@ namespace fsdit {
 // of the work it launches (host arithmetic; nothing is read back until stop).
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
-  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_COUNT
+  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);

@@ -6,3 +6,4 @@
 #include "gemm_tc.cu"
 #include "attn_tc.cu"
 #include "noalloc.cu"
+#include "history.cu"

@@ -109,9 +109,59 @@ def case_memory(a):
     return res
 
 
+def case_chunk(a):
+    """One steady-state long-video chunk of the 42-layer Flash backbone: the
+    6x34x60 target (boundary + 5 future latents) plus a full 11-frame history
+    (4,140 rows), 3 evaluations, replayed from a CUDA graph."""
+    w = S.WORKLOADS["flash_backbone_6x34x60"]
+    T, H, W = w.grid
+    layers, io = S.make_weights(w, device="cuda")
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights(l) for l in layers], api.IOWeights(io), w.compress)
+    inp = S.make_inputs(w, device="cuda")
+    lv = api.LongVideo(bb, w.grid, w.n_text, w.n_audio, w.video_ch)
+    g = torch.Generator(device="cuda").manual_seed(8)
+    lv.store.push(torch.randn(21 * H * W, w.video_ch, generator=g, device="cuda"))
+    seq, vl, has_b, base = lv.prepare()
+    n_grid, hw = T * H * W, H * W
+    vl[:n_grid].copy_(inp["video_lat"][:n_grid])
+    lv.store.copy_frame(base, vl[:hw])
+    v0, a0 = vl.clone(), inp["audio_lat"].clone()
+    al = a0.clone()
+
+    def step():
+        vl.copy_(v0)
+        al.copy_(a0)
+        bb.sample(seq, w.video_clock, w.audio_clock, vl, inp["text_emb"], al)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    ms = time_it(graph.replay, a.iters, a.warmup)
+    del graph
+    plan, n = lv.store.plan(base)
+    rows = lv.store.rows(plan, n)
+    lat = torch.empty(rows, w.video_ch, device="cuda")
+    pos = torch.empty(rows, 3, dtype=torch.int32, device="cuda")
+    g_ms = time_it(lambda: lv.store.gather(plan, n, lat, pos), 50, 5)
+    tokens = seq.n_tokens
+    A, Hd, F = w.attn_dim, w.hidden, w.ffn
+
+    def layer_flops(n):  # projections 2n(3AH + AH + 2HF) + attention 4n^2 A
+        return 2.0 * n * (4 * A * Hd + 2 * Hd * F) + 4.0 * n * n * A
+
+    per_eval = sum(layer_flops(seq.n_compressed if c else tokens) for c in w.compress)
+    tflop = per_eval * w.n_evals / 1e12
+    return {"case": "chunk", "tflop_per_chunk": tflop, "tflops": tflop / ms * 1e3, "workload": "flash_chunk_6x34x60_history11", "history_rows": rows, "tokens": tokens,
+            "compressed_tokens": seq.n_compressed, "ms_per_chunk": ms,
+            "tokens_per_s": tokens * w.n_evals / ms * 1e3, "new_frames_per_s": 17 / ms * 1e3,
+            "gather_ms": g_ms, "gather_gbs": rows * (w.video_ch * 8 + 12) / g_ms / 1e6}
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("case", choices=["attention", "gemm", "block", "memory"])
+    p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk"])
     p.add_argument("--n", type=int, default=12560)
     p.add_argument("--heads", type=int, default=56)
     p.add_argument("--M", type=int, default=12560)
@@ -125,7 +175,7 @@ def main():
     B.build()
     L.load()
     res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
-           "memory": case_memory}[a.case](a)
+           "memory": case_memory, "chunk": case_chunk}[a.case](a)
     api.device_error()
     print(json.dumps(res), flush=True)
 

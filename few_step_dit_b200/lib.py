@@ -57,6 +57,19 @@ class Tokens(C.Structure):
                 ("n_keep", C.c_int), ("near_idx", C.c_void_p)]
 
 
+class HistoryEntry(C.Structure):
+    _fields_ = [("frame", C.c_int), ("stride", C.c_int)]
+
+
+class HistoryStore(C.Structure):
+    _fields_ = [("frames", C.c_void_p), ("capacity", C.c_int), ("H", C.c_int), ("W", C.c_int),
+                ("C", C.c_int), ("n_frames", C.c_int)]
+
+
+HISTORY_MAX_ENTRIES = 11
+HISTORY_MIN_SLOTS = 12
+
+
 class ProfEntry(C.Structure):
     _fields_ = [("name", C.c_char * 32), ("scopes", C.c_int), ("launches", C.c_int),
                 ("ms", C.c_double), ("flops", C.c_double), ("bytes", C.c_double)]
@@ -92,6 +105,14 @@ _SIGS = {
     "dit_flow_sample": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(C.c_uint8),
                              C.POINTER(IOWeights), C.POINTER(Tokens), _I, C.POINTER(_F),
                              C.POINTER(_F), _P, _P, _P, _P, C.c_size_t, _P]),
+    "fsdit_history_bytes": (C.c_size_t, [_I, _I, _I, _I]),
+    "fsdit_history_init": (_I, [C.POINTER(HistoryStore), _P, _I, _I, _I, _I]),
+    "fsdit_history_push": (_I, [C.POINTER(HistoryStore), _P, _I, _P]),
+    "fsdit_history_plan": (_I, [_I, C.POINTER(HistoryEntry), _I]),
+    "fsdit_history_rows": (_I, [C.POINTER(HistoryEntry), _I, _I, _I]),
+    "fsdit_history_gather": (_I, [C.POINTER(HistoryStore), C.POINTER(HistoryEntry), _I, _P, _I, _P, _P]),
+    "fsdit_history_copy_frame": (_I, [C.POINTER(HistoryStore), _I, _P, _P]),
+    "fsdit_chunk_tags": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
 }
 
 _lib = None

@@ -319,6 +319,89 @@ FSDIT_API fsdit_status dit_block_forward_noalloc(const fsdit_dims* dims, const f
                                                  const fsdit_tokens* tok, const float* x_in, float* x_out,
                                                  fsdit_stream_t stream);
 
+/* ------------------------------------------------------------------ long video
+ * Chunked generation with a bounded, multi-stride history ([tokendh] section
+ * "长视频生成：怎么记住十分钟前发生的事"; [PaperDaily] section 三).  A chunk's
+ * target grid is T latent frames: frame 0 is the boundary latent (the last
+ * latent of the video so far; clean and never updated), frames 1..T-1 are new.
+ * Its history is made of latent frames before the boundary: frame 0 of the
+ * video at full resolution, the two newest at spatial stride 2 and at most
+ * eight before those at stride 4 (rows and columns that are multiples of the
+ * stride); frames in between are dropped.  History rows are clean video
+ * conditions at their original (t, h, w) and sit after the target grid rows
+ * (they are not token-compressed).  The first chunk has no boundary and no
+ * history. */
+
+#define FSDIT_HISTORY_MAX_ENTRIES 11 /* 1 full + 8 stride-4 + 2 stride-2 frames */
+#define FSDIT_HISTORY_MIN_SLOTS 12   /* frame 0, the 10 newest history frames, the boundary */
+
+/* One frame of a history plan, in time order. */
+typedef struct {
+  int frame;  /* index of the latent frame in the video (0 = first) */
+  int stride; /* spatial stride: 1, 2 or 4 */
+} fsdit_history_entry;
+
+/* The frame store: caller-owned device memory of `capacity` latent frames,
+ * each [H][W][C] fp32 (the video-latent layout of fsdit_tokens' video rows).
+ * Frame 0 stays in slot 0; frame i >= 1 goes to slot 1 + (i - 1) % (capacity
+ * - 1), so with capacity >= FSDIT_HISTORY_MIN_SLOTS every frame a plan names
+ * is still resident.  The struct is plain data; the library keeps no state. */
+typedef struct {
+  float* frames;  /* device, capacity * H * W * C floats, 16-byte aligned */
+  int capacity, H, W, C;
+  int n_frames;   /* latent frames pushed so far */
+} fsdit_history_store;
+
+/* Bytes of a store's frame memory. */
+FSDIT_API size_t fsdit_history_bytes(int capacity, int H, int W, int C);
+
+/* Set up `s` over caller memory `frames` (no device work).  Errors:
+ * FSDIT_E_NULL, FSDIT_E_SHAPE (capacity < FSDIT_HISTORY_MIN_SLOTS or a
+ * non-positive size), FSDIT_E_ALIGN. */
+FSDIT_API fsdit_status fsdit_history_init(fsdit_history_store* s, float* frames, int capacity, int H, int W,
+                                          int C);
+
+/* Append `n` latent frames (device, contiguous [n][H][W][C] fp32) to the
+ * video: asynchronous device copies on `stream`, then s->n_frames += n. */
+FSDIT_API fsdit_status fsdit_history_push(fsdit_history_store* s, const float* frames, int n,
+                                          fsdit_stream_t stream);
+
+/* Host: the history plan of a chunk whose boundary is frame `n_before` (the
+ * frames 0 .. n_before-1 come before it).  Writes at most `max_entries`
+ * entries to `out` and returns how many (0 .. FSDIT_HISTORY_MAX_ENTRIES), or
+ * -1 when n_before < 0 or `out` is too small. */
+FSDIT_API int fsdit_history_plan(int n_before, fsdit_history_entry* out, int max_entries);
+
+/* Host: history rows of a plan for an H x W frame. */
+FSDIT_API int fsdit_history_rows(const fsdit_history_entry* plan, int n_plan, int H, int W);
+
+/* Gather the plan's rows from the store: row r of the output is one (frame,
+ * h, w) of the plan, frame by frame in plan order, each frame row-major at
+ * its stride.  lat [rows][ld_lat] fp32 (C values written per row; ld_lat >=
+ * C) and pos [rows][3] int32 = (frame, h, w), both device.  Errors:
+ * FSDIT_E_SHAPE when a planned frame is not resident (never pushed, or
+ * overwritten), a stride is not 1, 2 or 4, or n_plan is out of range. */
+FSDIT_API fsdit_status fsdit_history_gather(const fsdit_history_store* s, const fsdit_history_entry* plan,
+                                            int n_plan, float* lat, int ld_lat, int32_t* pos,
+                                            fsdit_stream_t stream);
+
+/* Copy resident frame `frame` ([H][W][C] fp32) to device memory `dst`
+ * (e.g. the boundary slot of the next chunk's latents). */
+FSDIT_API fsdit_status fsdit_history_copy_frame(const fsdit_history_store* s, int frame, float* dst,
+                                                fsdit_stream_t stream);
+
+/* Host: row tags of one chunk, the layout fsdit_tokens expects: [target grid
+ * T x H x W at t = base + 0 .. T-1 | n_hist history rows | n_text text |
+ * n_audio audio].  Grid rows: video modality, time id 1, updated, except the
+ * boundary frame 0 when has_boundary (time id 0, not updated).  History rows:
+ * video modality, time id 0, not updated, pos left untouched (the gather
+ * writes it).  Text rows: time id 0, pos (0,0,0).  Audio rows: time id 2,
+ * updated, pos (floor(j T / n_audio) + base, 0, 0).  Host arrays of n =
+ * T*H*W + n_hist + n_text + n_audio entries (pos: 3n). */
+FSDIT_API fsdit_status fsdit_chunk_tags(int T, int H, int W, int base, int has_boundary, int n_hist, int n_text,
+                                        int n_audio, uint8_t* modality, uint8_t* time_id, uint8_t* out_mask,
+                                        int32_t* pos);
+
 #ifdef __cplusplus
 }
 #endif
