@@ -19,16 +19,17 @@ Sources (web write-ups of arXiv 2609.15863, "LynnReal-Omni"):
 * [tokendh] section "长视频生成：怎么记住十分钟前发生的事" (boundary frame,
   bounded multi-stride history).
 
-Modules: ``dit.py`` (block, compression, stack, flow-matching sampler) and
+Modules: ``dit.py`` (block, compression, stack, flow-matching sampler),
 ``long_video.py`` (chunked generation with the bounded history; import it as
-``oracle.long_video``).
+``oracle.long_video``) and ``fp8.py`` (E4M3 block projections; ``oracle.fp8``).
 
 Every floating-point step runs in float64.  Where the pages leave a step open
 the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
 
 Parity status per function: everything in ``dit.py`` is pinned by the CPU
 tests in ``tests/test_oracle_pins.py`` and everything in ``long_video.py`` by
-``tests/test_oracle_long_video.py``, except the conventions that are pure
+``tests/test_oracle_long_video.py``, everything in ``fp8.py`` by
+``tests/test_oracle_fp8.py``, except the conventions that are pure
 definitions (weight init, time-embedding MLP, bias placement); those are
 "parity unpinned" in the sense that no page fixes them, so the GPU path is
 compared against this oracle's definition of them.
