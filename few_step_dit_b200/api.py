@@ -27,27 +27,74 @@ def dtype_code(t_dtype):
 
 
 def make_dims(hidden, heads, ffn, dtype, head_dim=128, rope_split=(32, 48, 48), rms_eps=1e-6,
-              rope_theta=10000.0):
+              rope_theta=10000.0, proj_fp8=False):
     d = L.Dims()
     d.hidden, d.heads, d.head_dim, d.ffn = hidden, heads, head_dim, ffn
     d.rope_split[:] = list(rope_split)
     d.rms_eps, d.rope_theta = rms_eps, rope_theta
     d.dtype = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    d.proj_fp8 = int(bool(proj_fp8))
     return d
 
 
-def dims_of(w):
+def dims_of(w, proj_fp8=False):
     """Dims of a synthetic Workload."""
     return make_dims(w.hidden, w.heads, w.ffn, L.F32 if w.dtype == "f32" else L.BF16,
-                     w.head_dim, w.rope_split, w.rms_eps, w.rope_theta)
+                     w.head_dim, w.rope_split, w.rms_eps, w.rope_theta, proj_fp8)
 
 
 class BlockWeights:
-    """Device weights of one block (dict of tensors) and their C struct."""
+    """Device weights of one block (dict of tensors) and their C struct.  For
+    E4M3 projections the four projection weights are uint8 code tensors and
+    s_qkv, s_o, s_1, s_2 their scales (see quantize_block_weights)."""
 
     def __init__(self, tensors: dict):
         self.tensors = {k: v.contiguous() for k, v in tensors.items()}
-        self.struct = L.BlockWeights(*[self.tensors[k].data_ptr() for k in L.BLOCK_FIELDS])
+        ptrs = [self.tensors[k].data_ptr() for k in L.BLOCK_FIELDS]
+        ptrs += [self.tensors[k].data_ptr() if k in self.tensors else None for k in L.BLOCK_SCALE_FIELDS]
+        self.struct = L.BlockWeights(*ptrs)
+
+
+_PROJ = (("w_qkv", "s_qkv"), ("w_o", "s_o"), ("w_1", "s_1"), ("w_2", "s_2"))
+
+
+def quantize_rows(a, stream=None):
+    """Per-row E4M3 codes (uint8) and fp32 scales of a [rows, cols] fp32 or bf16 matrix."""
+    rows, cols = a.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device=a.device)
+    s = torch.empty(max(rows, 1), dtype=torch.float32, device=a.device)
+    L.call("fsdit_quantize_rows", L.ptr(a), dtype_code(a.dtype), rows, cols, L.ptr(q), L.ptr(s), _stream(stream))
+    return q, s[:rows]
+
+
+def quantize_block_weights(tensors: dict, stream=None):
+    """The same block with its four projection weights quantized per output
+    channel (E4M3 codes + scales), ready for dims with proj_fp8."""
+    out = dict(tensors)
+    for w, s in _PROJ:
+        out[w], out[s] = quantize_rows(tensors[w].contiguous(), stream)
+    return out
+
+
+def rmsnorm_quant(x, g, eps=1e-6, stream=None):
+    rows, hidden = x.shape
+    q = torch.empty(rows, hidden, dtype=torch.uint8, device=x.device)
+    s = torch.empty(max(rows, 1), dtype=torch.float32, device=x.device)
+    L.call("fsdit_rmsnorm_quant", L.ptr(x), L.ptr(g), rows, hidden, float(eps), L.ptr(q), L.ptr(s),
+           _stream(stream))
+    return q, s[:rows]
+
+
+def linear_fp8(dims, qa, sa, qw, sw, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, stream=None):
+    """E4M3 projection: epilogue((qa qw^T) * sa[row] * sw[col] + b)."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        od = torch.float32 if epilogue in (L.EPI_RESIDUAL, L.EPI_BIAS_F32) else torch.bfloat16
+        out = torch.empty(M, N, dtype=od, device=qa.device)
+    L.call("fsdit_linear_fp8", C.byref(dims), L.ptr(qa), L.ptr(sa), L.ptr(qw), L.ptr(sw), L.ptr(b), L.ptr(out),
+           L.ptr(resid), L.ptr(pos), M, N, K, epilogue, _stream(stream))
+    return out
 
 
 class IOWeights:

@@ -15,7 +15,9 @@ namespace fsdit {
 static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "gemm_gelu", "gemm_bias_f32",
                                            "gemm_bias",     "attention",     "rmsnorm_cast", "gather",
                                            "broadcast",     "embed",         "time_mlp",  "heads",
-                                           "euler",         "keep_map",  "rope_table", "history_gather"};
+                                           "euler",         "keep_map",  "rope_table", "history_gather",
+                                           "quantize",      "gemm_fp8_qkv_rope", "gemm_fp8_residual",
+                                           "gemm_fp8_gelu"};
 struct Prof {
   bool on = false;
   int used = 0;
@@ -145,6 +147,10 @@ static fsdit_status check_dims(const fsdit_dims* d) {
     set_error("dims: rms_eps must be >= 0 and rope_theta > 1");
     return FSDIT_E_SHAPE;
   }
+  if (d->proj_fp8 != 0 && (d->proj_fp8 != 1 || d->dtype != FSDIT_BF16)) {
+    set_error("dims.proj_fp8 must be 0, or 1 with dtype FSDIT_BF16");
+    return FSDIT_E_DTYPE;
+  }
   return FSDIT_OK;
 }
 
@@ -164,6 +170,8 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.s0 = d->rope_split[0];
   e.s1 = d->rope_split[1];
   e.log2_theta = log2f(d->rope_theta);
+  e.row_scale = nullptr;
+  e.col_scale = nullptr;
   return e;
 }
 
@@ -178,6 +186,20 @@ fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, co
   ProfScope ps(prof_cls >= 0 ? prof_cls : cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);
   if (d->dtype == FSDIT_BF16) return launch_linear_tc(a, w, ep, M, N, K, st);
   return launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
+}
+
+fsdit_status launch_linear_fp8(const fsdit_dims* d, const uint8_t* qa, const void* qw, const EpiParams& ep, int M,
+                               int N, int K, cudaStream_t st) {
+  if (M <= 0) return FSDIT_OK;
+  const int cls = ep.epi == FSDIT_EPI_QKV_ROPE ? PC_GEMM_FP8_QKV
+                  : ep.epi == FSDIT_EPI_GELU   ? PC_GEMM_FP8_GELU
+                                               : PC_GEMM_FP8_RESID;
+  const double out_b = (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32) ? 4.0 : 2.0;
+  const double by = (double)M * K + (double)N * K + (double)M * N * out_b +
+                    (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
+  ProfScope ps(cls, 1, 2.0 * M * N * K, by, st);
+  (void)d;
+  return launch_linear_fp8_tc(qa, (const uint8_t*)qw, ep, M, N, K, st);
 }
 
 fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n, cudaStream_t st) {
@@ -198,14 +220,16 @@ struct Carve {
   }
 };
 
-struct BlockWs {
-  float* xc;       // [n_c, hidden] compressed residual (compressed mode)
-  int32_t* posc;   // [n_c, 3]
-  void* xn;        // [n, max(hidden, attn)] GEMM operand (normalized x / attention output)
-  void* qkv;       // [n, 3 attn]
-  void* u;         // [n, ffn]
-  float2* rope;    // [n, head_dim/2] (cos, sin) table of the rows' positions
-  float2* rope_c;  // stack only: table of the compressed rows
+struct BlockWs {  // every buffer null until a carve sets it
+  float* xc = nullptr;       // [n_c, hidden] compressed residual (compressed mode)
+  int32_t* posc = nullptr;   // [n_c, 3]
+  void* xn = nullptr;        // [n, max(hidden, attn)] GEMM operand (normalized x / attention output)
+  void* qkv = nullptr;       // [n, 3 attn]
+  void* u = nullptr;         // [n, ffn]
+  float2* rope = nullptr;    // [n, head_dim/2] (cos, sin) table of the rows' positions
+  float2* rope_c = nullptr;  // stack only: table of the compressed rows
+  uint8_t* q8 = nullptr;     // FP8 projections: [n, max(hidden, attn, ffn)] E4M3 operand
+  float* sa = nullptr;       //                  [n] its row scales
 };
 
 static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, bool compressed) {
@@ -219,6 +243,13 @@ static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, b
   w.u = c.take((size_t)n * d->ffn * dsize(d->dtype));
   w.rope = (float2*)c.take((size_t)n * (d->head_dim / 2) * sizeof(float2));
   w.rope_c = nullptr;
+  w.q8 = nullptr;
+  w.sa = nullptr;
+  if (d->proj_fp8) {
+    const int k8 = wide > d->ffn ? wide : d->ffn;
+    w.q8 = (uint8_t*)c.take((size_t)n * k8);
+    w.sa = (float*)c.take((size_t)n * 4);
+  }
   return w;
 }
 
@@ -229,8 +260,46 @@ static fsdit_status rope_table(const fsdit_dims* d, const int32_t* pos, int rows
 }
 
 // x_in -> x_out over n rows; `rope` is the (cos, sin) table of the rows' positions.
+// E4M3 projections: each GEMM operand is quantized per row (RMSNorm fused with
+// it for the QKV and FFN-up inputs; a separate pass over the bf16 attention
+// and GELU outputs for the O and FFN-down inputs); the weights carry their
+// per-output-channel scales; the epilogue dequantizes before the bias.
+static fsdit_status block_body_fp8(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
+                                   const int32_t* pos, const float2* rope, int n, const BlockWs& ws,
+                                   cudaStream_t st) {
+  const int H = d->hidden, F = d->ffn, A = attn_dim(d);
+  if (ws.q8 == nullptr || ws.sa == nullptr) {
+    set_error("FP8 projections: the workspace has no quantized-operand buffers");
+    return FSDIT_E_WORKSPACE;
+  }
+  auto scaled = [&](EpiParams e, const float* col_scale) {
+    e.row_scale = ws.sa;
+    e.col_scale = col_scale;
+    return e;
+  };
+  FS_TRY(launch_rmsnorm_quant(x_in, w->g_attn, n, H, d->rms_eps, ws.q8, ws.sa, st));
+  EpiParams qkv_ep = scaled(make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos), w->s_qkv);
+  qkv_ep.rope_cs = rope;
+  FS_TRY(launch_linear_fp8(d, ws.q8, w->w_qkv, qkv_ep, n, 3 * A, H, st));
+  FS_TRY(launch_attention(d, ws.qkv, ws.xn, n, st));
+  FS_TRY(launch_quant_rows(ws.xn, FSDIT_BF16, n, A, ws.q8, ws.sa, st));
+  FS_TRY(launch_linear_fp8(d, ws.q8, w->w_o,
+                           scaled(make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), w->s_o), n, H, A,
+                           st));
+  FS_TRY(launch_rmsnorm_quant(x_out, w->g_ffn, n, H, d->rms_eps, ws.q8, ws.sa, st));
+  FS_TRY(launch_linear_fp8(d, ws.q8, w->w_1, scaled(make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr),
+                                                    w->s_1),
+                           n, F, H, st));
+  FS_TRY(launch_quant_rows(ws.u, FSDIT_BF16, n, F, ws.q8, ws.sa, st));
+  FS_TRY(launch_linear_fp8(d, ws.q8, w->w_2,
+                           scaled(make_ep(d, FSDIT_EPI_RESIDUAL, w->b_2, x_out, H, x_out, nullptr), w->s_2), n, H, F,
+                           st));
+  return FSDIT_OK;
+}
+
 static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
                                const int32_t* pos, const float2* rope, int n, const BlockWs& ws, cudaStream_t st) {
+  if (d->proj_fp8) return block_body_fp8(d, w, x_in, x_out, pos, rope, n, ws, st);
   const int H = d->hidden, F = d->ffn, A = attn_dim(d);
   FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
   EpiParams qkv_ep = make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos);
@@ -246,8 +315,14 @@ static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w
   return FSDIT_OK;
 }
 
-static fsdit_status check_block_weights(const fsdit_block_weights* w) {
+static fsdit_status check_block_weights(const fsdit_dims* d, const fsdit_block_weights* w) {
   FS_TRY(need(w, "weights"));
+  if (d->proj_fp8) {
+    FS_TRY(need(w->s_qkv, "s_qkv"));
+    FS_TRY(need(w->s_o, "s_o"));
+    FS_TRY(need(w->s_1, "s_1"));
+    FS_TRY(need(w->s_2, "s_2"));
+  }
   FS_TRY(need(w->w_qkv, "w_qkv"));
   FS_TRY(need(w->b_qkv, "b_qkv"));
   FS_TRY(need(w->w_o, "w_o"));
@@ -413,6 +488,13 @@ static size_t stack_carve(Carve& c, const fsdit_dims* d, const fsdit_io_weights*
   w.u = c.take((size_t)N * d->ffn * dsize(d->dtype));
   w.rope = (float2*)c.take((size_t)N * (d->head_dim / 2) * sizeof(float2));
   w.rope_c = comp ? (float2*)c.take((size_t)n_c * (d->head_dim / 2) * sizeof(float2)) : nullptr;
+  w.q8 = nullptr;
+  w.sa = nullptr;
+  if (d->proj_fp8) {
+    const int k8 = wide > d->ffn ? wide : d->ffn;
+    w.q8 = (uint8_t*)c.take((size_t)N * k8);
+    w.sa = (float*)c.take((size_t)N * 4);
+  }
   *bw = w;
   return c.off;
 }
@@ -519,6 +601,86 @@ fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, 
   return launch_linear(dims, a, w, ep, M, N, K, (cudaStream_t)stream);
 }
 
+
+
+fsdit_status fsdit_quantize_rows(const void* a, int dtype, int rows, int cols, uint8_t* q, float* s,
+                                 fsdit_stream_t stream) {
+  FS_TRY(need(a, "a"));
+  FS_TRY(need(q, "q"));
+  FS_TRY(need(s, "s"));
+  if (dtype != FSDIT_F32 && dtype != FSDIT_BF16) {
+    set_error("quantize_rows: bad dtype %d", dtype);
+    return FSDIT_E_DTYPE;
+  }
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) {
+    set_error("quantize_rows: need rows >= 0, cols > 0, cols %% 16 == 0 (got %d %d)", rows, cols);
+    return FSDIT_E_SHAPE;
+  }
+  if (!aligned16(a) || !aligned16(q)) {
+    set_error("quantize_rows: a and q must be 16-byte aligned");
+    return FSDIT_E_ALIGN;
+  }
+  return launch_quant_rows(a, dtype, rows, cols, q, s, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_rmsnorm_quant(const float* x, const void* g, int rows, int hidden, float eps, uint8_t* q, float* s,
+                                 fsdit_stream_t stream) {
+  FS_TRY(need(x, "x"));
+  FS_TRY(need(g, "g"));
+  FS_TRY(need(q, "q"));
+  FS_TRY(need(s, "s"));
+  if (rows < 0 || hidden <= 0 || hidden % 64 != 0 || hidden > 8192 || !(eps >= 0.f)) {
+    set_error("rmsnorm_quant: need rows >= 0, hidden %% 64 == 0, hidden <= 8192, eps >= 0");
+    return FSDIT_E_SHAPE;
+  }
+  if (!aligned16(x) || !aligned16(q)) {
+    set_error("rmsnorm_quant: x and q must be 16-byte aligned");
+    return FSDIT_E_ALIGN;
+  }
+  return launch_rmsnorm_quant(x, g, rows, hidden, eps, q, s, (cudaStream_t)stream);
+}
+
+fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* qa, const float* sa, const uint8_t* qw,
+                              const float* sw, const void* b, void* out, const float* resid, const int32_t* pos, int M,
+                              int N, int K, int epilogue, fsdit_stream_t stream) {
+  FS_TRY(check_dims(dims));
+  if (dims->dtype != FSDIT_BF16) {
+    set_error("linear_fp8: dims.dtype must be FSDIT_BF16 (bias, outputs)");
+    return FSDIT_E_DTYPE;
+  }
+  FS_TRY(need(qa, "qa"));
+  FS_TRY(need(sa, "sa"));
+  FS_TRY(need(qw, "qw"));
+  FS_TRY(need(sw, "sw"));
+  FS_TRY(need(b, "b"));
+  FS_TRY(need(out, "out"));
+  if (M < 0 || N <= 0 || K <= 0 || K % 16 != 0 || N % 32 != 0) {
+    set_error("linear_fp8: need M >= 0, N %% 32 == 0, K %% 16 == 0 (got %d %d %d)", M, N, K);
+    return FSDIT_E_SHAPE;
+  }
+  if (epilogue < FSDIT_EPI_BIAS || epilogue > FSDIT_EPI_RESIDUAL) {
+    set_error("linear_fp8: unknown epilogue %d", epilogue);
+    return FSDIT_E_SHAPE;
+  }
+  if (epilogue == FSDIT_EPI_RESIDUAL) FS_TRY(need(resid, "resid"));
+  if (epilogue == FSDIT_EPI_QKV_ROPE) {
+    FS_TRY(need(pos, "pos"));
+    if (N != 3 * attn_dim(dims)) {
+      set_error("linear_fp8: the RoPE epilogue needs N == 3*heads*head_dim");
+      return FSDIT_E_SHAPE;
+    }
+  }
+  if (!aligned16(qa) || !aligned16(qw) || !aligned16(sw) || !aligned16(b) || !aligned16(out) ||
+      (resid != nullptr && !aligned16(resid))) {
+    set_error("linear_fp8: qa, qw, sw, b, out and resid must be 16-byte aligned");
+    return FSDIT_E_ALIGN;
+  }
+  EpiParams ep = make_ep(dims, epilogue, b, out, N, resid, pos);
+  ep.row_scale = sa;
+  ep.col_scale = sw;
+  return launch_linear_fp8(dims, qa, qw, ep, M, N, K, (cudaStream_t)stream);
+}
+
 fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n, fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));
   FS_TRY(need(qkv, "qkv"));
@@ -534,7 +696,7 @@ fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_block_weights
                                const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
                                fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));
-  FS_TRY(check_block_weights(w));
+  FS_TRY(check_block_weights(dims, w));
   FS_TRY(check_tokens(tok, false));
   FS_TRY(need(x_in, "x_in"));
   FS_TRY(need(x_out, "x_out"));
@@ -661,7 +823,7 @@ static fsdit_status check_stack_args(const fsdit_dims* dims, int n_layers, const
     set_error("stack: n_layers >= 0 and host arrays layers / layer_compress are required");
     return FSDIT_E_NULL;
   }
-  for (int l = 0; l < n_layers; ++l) FS_TRY(check_block_weights(&layers[l]));
+  for (int l = 0; l < n_layers; ++l) FS_TRY(check_block_weights(dims, &layers[l]));
   if (n_times <= 0 || n_times > 8) {
     set_error("stack: 1 <= n_times <= 8");
     return FSDIT_E_SHAPE;

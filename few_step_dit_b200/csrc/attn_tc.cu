@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < BKV; c += 2) {
         float x0, x1, p0, p1;
         f2_split(f2_fma(f2(s[c], s[c + 1]), scale2, negm2), x0, x1);
-        if (EMU_EVERY > 0 && (c >> 1) % EMU_EVERY == EMU_EVERY - 1) {
+        if (EMU_EVERY > 0 && (c >> 1) % (EMU_EVERY > 0 ? EMU_EVERY : 1) == EMU_EVERY - 1) {
           exp2_poly_pair(x0, x1, p0, p1);
         } else {
           p0 = ex2(x0);

@@ -66,12 +66,19 @@ struct EpiParams {
   int rope_cols;        // columns [0, rope_cols) are rotated
   int head_dim, s0, s1;
   float log2_theta;
+  const float* row_scale;  // [M] or null: accumulators are multiplied by
+  const float* col_scale;  // row_scale[row] * col_scale[col] (FP8 dequantization) before the bias
 };
 
 // Apply the epilogue to `cnt` consecutive columns [col, col+cnt) of one row.
 // v[] holds the fp32 accumulators; cnt is even and col is even.
 template <typename TW, int CNT>
 __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int col, float* v) {
+  if (p.col_scale != nullptr) {
+    const float rs = p.row_scale[row];
+#pragma unroll
+    for (int i = 0; i < CNT; ++i) v[i] *= rs * p.col_scale[col + i];
+  }
   const TW* bias = reinterpret_cast<const TW*>(p.bias);
 #pragma unroll
   for (int i = 0; i < CNT; ++i) v[i] += ld_f32<TW>(bias + col + i);
@@ -155,6 +162,8 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
 struct Epi32Pre {
   uint4 bias[4];    // 32 bf16 bias values (the same for every row)
   float4 extra[8];  // QKV_ROPE: 16 (cos, sin) pairs; RESIDUAL: 32 fp32 residual values
+  float4 cscale[8]; // FP8 dequantization: 32 column scales (same for every row)
+  float rscale;     //                     and this row's scale
 };
 
 // GELU (tanh form) with the hardware tanh approximation (relative error about
@@ -176,6 +185,12 @@ __device__ __forceinline__ void epi32_prefetch(const EpiParams& p, int row, int 
   const uint4* b = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(p.bias) + col);
 #pragma unroll
   for (int i = 0; i < 4; ++i) e.bias[i] = __ldg(b + i);
+  if (p.col_scale != nullptr) {
+    const float4* cs = reinterpret_cast<const float4*>(p.col_scale + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e.cscale[i] = __ldg(cs + i);
+    e.rscale = __ldg(p.row_scale + row);
+  }
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
     if (col < p.rope_cols && p.rope_cs != nullptr) {
       const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (size_t)row * (p.head_dim >> 1) +
@@ -191,6 +206,15 @@ __device__ __forceinline__ void epi32_prefetch(const EpiParams& p, int row, int 
 }
 
 __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col, float* v, const Epi32Pre& e) {
+  if (p.col_scale != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[4 * i] *= e.rscale * e.cscale[i].x;
+      v[4 * i + 1] *= e.rscale * e.cscale[i].y;
+      v[4 * i + 2] *= e.rscale * e.cscale[i].z;
+      v[4 * i + 3] *= e.rscale * e.cscale[i].w;
+    }
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&e.bias[i]);
@@ -259,7 +283,8 @@ namespace fsdit {
 // of the work it launches (host arithmetic; nothing is read back until stop).
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
-  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_COUNT
+  PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_QUANT,
+  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);
@@ -280,6 +305,13 @@ fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep,
                               int K, cudaStream_t st);
 fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n,
                               cudaStream_t st);
+fsdit_status launch_linear_fp8(const fsdit_dims* d, const uint8_t* qa, const void* qw, const EpiParams& ep, int M,
+                               int N, int K, cudaStream_t st);
+fsdit_status launch_linear_fp8_tc(const uint8_t* qa, const uint8_t* qw, const EpiParams& ep, int M, int N, int K,
+                                  cudaStream_t st);
+fsdit_status launch_quant_rows(const void* a, int dtype, int rows, int cols, uint8_t* q, float* s, cudaStream_t st);
+fsdit_status launch_rmsnorm_quant(const float* x, const void* g, int rows, int hidden, float eps, uint8_t* q,
+                                  float* s, cudaStream_t st);
 fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n, int heads,
                                    int hidden, cudaStream_t st);
 fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int attn,

@@ -1,0 +1,147 @@
+// FP8 (E4M3) quantization for the low-bit block projections ([PaperDaily]
+// section 二, third step: low-bit weights and activations, quantization fused
+// next to the normalization).
+//
+// One fp32 scale per row: s = amax / 448 (1 for an all-zero row) and codes
+// E4M3(v / s), round to nearest even, saturating; amax, the IEEE division and
+// the rounding happen in fp32.  Activations are quantized per token, weights
+// per output channel (rows of [N, K]).
+
+namespace fsdit {
+namespace q8 {
+
+constexpr float E4M3_MAX = 448.0f;
+
+// Two E4M3 codes, `lo` in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float m = 0.f;
+  const int nw = blockDim.x >> 5;
+  for (int i = 0; i < nw; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+__device__ __forceinline__ float row_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, E4M3_MAX) : 1.0f; }
+
+// 8 consecutive values as fp32.
+template <typename T> __device__ __forceinline__ void load8(const T* p, float* v);
+template <> __device__ __forceinline__ void load8<float>(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <> __device__ __forceinline__ void load8<bf16>(const bf16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// One 256-thread block per row: amax pass, then the codes (cols % 8 == 0).
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int cols, uint8_t* __restrict__ q,
+                                                         float* __restrict__ s) {
+  __shared__ float red[8];
+  const int r = blockIdx.x;
+  const T* ar = a + (size_t)r * cols;
+  float amax = 0.f;
+  for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
+    float v[8];
+    load8<T>(ar + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  }
+  const float sc = row_scale(block_max(amax, red));
+  if (threadIdx.x == 0) s[r] = sc;
+  uint8_t* qr = q + (size_t)r * cols;
+  for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
+    float v[8];
+    load8<T>(ar + c, v);
+    uint2 out;
+    out.x = (uint32_t)e4m3x2(__fdiv_rn(v[0], sc), __fdiv_rn(v[1], sc)) |
+            ((uint32_t)e4m3x2(__fdiv_rn(v[2], sc), __fdiv_rn(v[3], sc)) << 16);
+    out.y = (uint32_t)e4m3x2(__fdiv_rn(v[4], sc), __fdiv_rn(v[5], sc)) |
+            ((uint32_t)e4m3x2(__fdiv_rn(v[6], sc), __fdiv_rn(v[7], sc)) << 16);
+    *reinterpret_cast<uint2*>(qr + c) = out;
+  }
+}
+
+// RMSNorm of an fp32 row (gain bf16) fused with the quantization of its
+// output: y = x * rstd * g in fp32, kept in registers for the amax pass and
+// the codes (hidden <= 256 * 4 * RMS_MAXV, hidden % 4 == 0).
+__global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const float* __restrict__ x, const bf16* __restrict__ g,
+                                                            int hidden, float eps, uint8_t* __restrict__ q,
+                                                            float* __restrict__ s) {
+  __shared__ float red[8];
+  __shared__ float red2[8];
+  const int h4 = hidden >> 2;
+  const int r = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * hidden);
+  float4 v[RMS_MAXV];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < RMS_MAXV; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < h4) {
+      v[k] = xr[i];
+      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+    }
+  }
+  const float rstd = rsqrtf(block_sum(ss, red) / (float)hidden + eps);
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < RMS_MAXV; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < h4) {
+      const float4 gg = load_g4<bf16>(g + 4 * i);
+      v[k] = make_float4(v[k].x * rstd * gg.x, v[k].y * rstd * gg.y, v[k].z * rstd * gg.z, v[k].w * rstd * gg.w);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
+    }
+  }
+  const float sc = row_scale(block_max(amax, red2));
+  if (threadIdx.x == 0) s[r] = sc;
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + (size_t)r * hidden);
+#pragma unroll
+  for (int k = 0; k < RMS_MAXV; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < h4)
+      qr[i] = (uint32_t)e4m3x2(__fdiv_rn(v[k].x, sc), __fdiv_rn(v[k].y, sc)) |
+              ((uint32_t)e4m3x2(__fdiv_rn(v[k].z, sc), __fdiv_rn(v[k].w, sc)) << 16);
+  }
+}
+
+}  // namespace q8
+
+fsdit_status launch_quant_rows(const void* a, int dtype, int rows, int cols, uint8_t* q, float* s, cudaStream_t st) {
+  if (rows <= 0) return FSDIT_OK;
+  ProfScope ps(PC_QUANT, 1, 0.0, (double)rows * cols * (dtype == FSDIT_BF16 ? 2.0 : 4.0) * 2.0 + (double)rows * cols,
+               st);
+  if (dtype == FSDIT_BF16)
+    q8::quant_rows_kernel<bf16><<<rows, 256, 0, st>>>((const bf16*)a, cols, q, s);
+  else
+    q8::quant_rows_kernel<float><<<rows, 256, 0, st>>>((const float*)a, cols, q, s);
+  return cuda_check(cudaGetLastError(), "quant_rows_kernel");
+}
+
+fsdit_status launch_rmsnorm_quant(const float* x, const void* g, int rows, int hidden, float eps, uint8_t* q, float* s,
+                                  cudaStream_t st) {
+  if (rows <= 0) return FSDIT_OK;
+  ProfScope ps(PC_NORM, 1, 0.0, (double)rows * hidden * 5.0, st);
+  q8::rmsnorm_quant_kernel<<<rows, 256, 0, st>>>(x, (const bf16*)g, hidden, eps, q, s);
+  return cuda_check(cudaGetLastError(), "rmsnorm_quant_kernel");
+}
+
+}  // namespace fsdit

@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // per warp).
 namespace gemm2 {
 
-constexpr int BM = 256, BN = 256, BK = 64;
+constexpr int BM = 256, BN = 256, BK = 64;  // BK: bf16 elements per stage row (128 bytes)
+constexpr int BK8 = 128;                     // E4M3 elements per stage row (128 bytes)
 constexpr int HM = BM / 2, HN = BN / 2;  // per-CTA share of A rows and B rows
 constexpr int STAGES = 6;
 constexpr int A_BYTES = HM * BK * 2;
@@ -217,10 +218,15 @@ constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr int GROUP_N = 8;
 constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, 0);
+constexpr uint32_t IDESC_FP8 = ptx::idesc_e4m3(BM, BN);
 
+// FP8 = true: E4M3 operands (kind::f8f6f4, 32 K elements per MMA), the same
+// 128-byte stage rows; the epilogue applies the per-row / per-column scales.
+template <bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const gemm::Args args) {
+  constexpr int BKE = FP8 ? BK8 : BK;  // K elements per stage
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   const int num_tiles = args.tiles_m * args.tiles_n;
-  const int KB = (args.K + BK - 1) / BK;
+  const int KB = (args.K + BKE - 1) / BKE;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -284,8 +290,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sa = base + s * STAGE_BYTES;
           const uint32_t full = full0 + 8u * (uint32_t)s;
           if (rank == 0) mbar_expect_tx(FULL(s), 2 * STAGE_BYTES);
-          tma_load_2d_pair(sa, &tmA, kb * BK, row_a, full);
-          tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, row_b, full);
+          tma_load_2d_pair(sa, &tmA, kb * BKE, row_a, full);
+          tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BKE, row_b, full);
           last_s = s;
           last_ph = ph;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -316,10 +322,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(FULL(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + A_BYTES;
+          // four MMAs of 32 bytes of K each (16 bf16 or 32 E4M3 elements)
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_bf16_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC,
-                             (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (FP8)
+              mma_e4m3_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC_FP8,
+                               (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_bf16_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC,
+                               (kb | k) != 0 ? 1u : 0u);
+          }
           tc_commit_pair(EMPTY(s));
           tc_commit_pair(empty_peer0 + 8u * (uint32_t)s);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -390,8 +402,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 static std::once_flag g_encode_once;
 
-fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
-                            uint32_t box_rows, uint32_t box_cols) {
+// The driver's cuTensorMapEncodeTiled, looked up once.
+static fsdit_status encode_fn() {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
@@ -403,6 +415,12 @@ fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uin
     set_error("cuTensorMapEncodeTiled is not available from the driver");
     return FSDIT_E_CUDA;
   }
+  return FSDIT_OK;
+}
+
+fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                            uint32_t box_rows, uint32_t box_cols) {
+  FS_TRY(encode_fn());
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(row_stride_elems * 2)};
   cuuint32_t box[2] = {box_cols, box_rows};
@@ -420,16 +438,34 @@ fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uin
 
 // How many CTA pairs of tc_gemm_pair_kernel fit on the device at once
 // (0: the pair kernel cannot run, use the single-CTA kernel).
+fsdit_status make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride,
+                          uint32_t box_rows, uint32_t box_cols) {
+  FS_TRY(encode_fn());
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode_tiled(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled (u8) failed (%d) rows=%llu cols=%llu", (int)r, (unsigned long long)rows,
+              (unsigned long long)cols);
+    return FSDIT_E_CUDA;
+  }
+  return FSDIT_OK;
+}
+
 static int pair_clusters_resident() {
   static std::once_flag once;
   static int n = 0;
   std::call_once(once, [] {
-    if (cudaFuncSetAttribute(gemm2::tc_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemm2::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm2::tc_gemm_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) !=
-            cudaSuccess) {
-      (void)cudaGetLastError();
-      return;
+    for (auto fn : {gemm2::tc_gemm_pair_kernel<false>, gemm2::tc_gemm_pair_kernel<true>}) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return;
+      }
     }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
@@ -443,19 +479,21 @@ static int pair_clusters_resident() {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel, &cfg) == cudaSuccess) n = c;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel<false>, &cfg) == cudaSuccess) n = c;
     (void)cudaGetLastError();
   });
   return n;
 }
 
 static fsdit_status launch_linear_pair(const void* a, const void* w, const EpiParams& ep, int M, int N, int K,
-                                       int clusters, cudaStream_t st) {
+                                       int clusters, bool fp8, cudaStream_t st) {
   using namespace gemm2;
   CUtensorMap tmA, tmB;
-  fsdit_status s = make_tmap_bf16(&tmA, a, (uint64_t)M, (uint64_t)K, (uint64_t)K, HM, BK);
+  fsdit_status s = fp8 ? make_tmap_u8(&tmA, a, (uint64_t)M, (uint64_t)K, (uint64_t)K, HM, BK8)
+                       : make_tmap_bf16(&tmA, a, (uint64_t)M, (uint64_t)K, (uint64_t)K, HM, BK);
   if (s != FSDIT_OK) return s;
-  s = make_tmap_bf16(&tmB, w, (uint64_t)N, (uint64_t)K, (uint64_t)K, HN, BK);
+  s = fp8 ? make_tmap_u8(&tmB, w, (uint64_t)N, (uint64_t)K, (uint64_t)K, HN, BK8)
+          : make_tmap_bf16(&tmB, w, (uint64_t)N, (uint64_t)K, (uint64_t)K, HN, BK);
   if (s != FSDIT_OK) return s;
   gemm::Args args;
   args.M = M;
@@ -479,7 +517,20 @@ static fsdit_status launch_linear_pair(const void* a, const void* w, const EpiPa
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel, tmA, tmB, args), "tc_gemm_pair_kernel");
+  if (fp8)
+    return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<true>, tmA, tmB, args), "tc_gemm_pair_kernel<fp8>");
+  return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<false>, tmA, tmB, args), "tc_gemm_pair_kernel");
+}
+
+// E4M3 projection: always on pair tiles (their epilogue applies the scales).
+fsdit_status launch_linear_fp8_tc(const uint8_t* qa, const uint8_t* qw, const EpiParams& ep, int M, int N, int K,
+                                  cudaStream_t st) {
+  const int clusters = pair_clusters_resident();
+  if (clusters <= 0) {
+    set_error("linear_fp8: the CTA-pair GEMM cannot be made resident on this device");
+    return FSDIT_E_CUDA;
+  }
+  return launch_linear_pair(qa, qw, ep, M, N, K, clusters, true, st);
 }
 
 fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep, int M, int N, int K,
@@ -493,7 +544,7 @@ fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep,
                       (ep.rope_cs == nullptr || a16(ep.rope_cs)) && (ep.head_dim & (ep.head_dim - 1)) == 0;
   if (M > gemm2::HM && vec_ok) {
     const int clusters = pair_clusters_resident();
-    if (clusters > 0) return launch_linear_pair(a, w, ep, M, N, K, clusters, st);
+    if (clusters > 0) return launch_linear_pair(a, w, ep, M, N, K, clusters, false, st);
   }
   using namespace gemm;
   static std::once_flag attr_once;

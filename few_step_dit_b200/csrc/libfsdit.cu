@@ -2,6 +2,7 @@
 // every kernel live in one module, so no relocatable device code is needed.
 #include "api.cu"
 #include "elementwise.cu"
+#include "fp8.cu"
 #include "simt.cu"
 #include "gemm_tc.cu"
 #include "attn_tc.cu"

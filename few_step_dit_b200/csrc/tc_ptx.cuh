@@ -279,6 +279,23 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t cluster_bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
                : "memory");
 }
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0),
+// fp32 D, both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Pair MMA on E4M3 operands (32 K elements per instruction), fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Pair MMA, issued by one thread of cluster rank 0; descriptors are offsets
 // valid in both CTAs' shared memory, d_tmem a column of the pair allocation.
 __device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -297,5 +314,8 @@ __device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc
 // a (box_cols x box_rows) box and 128-byte swizzle (box_cols * 2 == 128).
 fsdit_status make_tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
                             uint32_t box_rows, uint32_t box_cols);
+// The same over a byte matrix (E4M3 codes); box_cols == 128.
+fsdit_status make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride,
+                          uint32_t box_rows, uint32_t box_cols);
 
 }  // namespace fsdit

@@ -32,16 +32,17 @@ class FsditError(RuntimeError):
 class Dims(C.Structure):
     _fields_ = [("hidden", C.c_int), ("heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
                 ("rope_split", C.c_int * 3), ("rms_eps", C.c_float), ("rope_theta", C.c_float),
-                ("dtype", C.c_int)]
+                ("dtype", C.c_int), ("proj_fp8", C.c_int)]
 
 
 BLOCK_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "w_1", "b_1", "w_2", "b_2", "g_attn", "g_ffn")
+BLOCK_SCALE_FIELDS = ("s_qkv", "s_o", "s_1", "s_2")  # per-output-channel scales of E4M3 projections
 IO_FIELDS = ("w_vin", "b_vin", "w_tin", "b_tin", "w_ain", "b_ain", "mod_emb", "w_t1", "b_t1",
              "w_t2", "b_t2", "g_out", "w_vout", "b_vout", "w_aout", "b_aout")
 
 
 class BlockWeights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in BLOCK_FIELDS]
+    _fields_ = [(n, C.c_void_p) for n in BLOCK_FIELDS + BLOCK_SCALE_FIELDS]
 
 
 class IOWeights(C.Structure):
@@ -105,6 +106,9 @@ _SIGS = {
     "dit_flow_sample": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(C.c_uint8),
                              C.POINTER(IOWeights), C.POINTER(Tokens), _I, C.POINTER(_F),
                              C.POINTER(_F), _P, _P, _P, _P, C.c_size_t, _P]),
+    "fsdit_quantize_rows": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "fsdit_rmsnorm_quant": (_I, [_P, _P, _I, _I, _F, _P, _P, _P]),
+    "fsdit_linear_fp8": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "fsdit_history_bytes": (C.c_size_t, [_I, _I, _I, _I]),
     "fsdit_history_init": (_I, [C.POINTER(HistoryStore), _P, _I, _I, _I, _I]),
     "fsdit_history_push": (_I, [C.POINTER(HistoryStore), _P, _I, _P]),

@@ -82,6 +82,9 @@ typedef struct {
   float rms_eps;    /* RMSNorm epsilon (1e-6) */
   float rope_theta; /* RoPE base (10000) */
   int dtype;        /* fsdit_dtype of weights and GEMM operands */
+  int proj_fp8;     /* 1: the four block projections run on FP8 E4M3 operands
+                       (dtype must be FSDIT_BF16; see "Low-bit projections"
+                       below); 0: they run in `dtype` */
 } fsdit_dims;
 
 /* Weights of one pre-norm DiT block (all (device), `dtype`); A = heads*128.
@@ -91,9 +94,14 @@ typedef struct {
  *   w_o   [hidden, A],   b_o [hidden]
  *   w_1   [ffn, hidden],     b_1 [ffn]
  *   w_2   [hidden, ffn],     b_2 [hidden]
- *   g_attn, g_ffn [hidden]   RMSNorm gains */
+ *   g_attn, g_ffn [hidden]   RMSNorm gains
+ * With dims.proj_fp8 = 1, w_qkv, w_o, w_1 and w_2 hold E4M3 codes (one byte
+ * each, same shapes) and s_qkv [3*A], s_o [hidden], s_1 [ffn], s_2 [hidden]
+ * their per-output-channel fp32 scales (fsdit_quantize_rows of the bf16
+ * weights); otherwise the s_* are unused (NULL). */
 typedef struct {
   const void *w_qkv, *b_qkv, *w_o, *b_o, *w_1, *b_1, *w_2, *b_2, *g_attn, *g_ffn;
+  const float *s_qkv, *s_o, *s_1, *s_2;
 } fsdit_block_weights;
 
 /* Embedding, timestep-MLP and output-head weights (all (device), `dtype`).
@@ -231,6 +239,36 @@ enum {
 FSDIT_API fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, const void* b,
                           void* out, const float* resid, const int32_t* pos, int M, int N, int K,
                           int epilogue, fsdit_stream_t stream);
+
+/* ------------------------------------------------------ low-bit projections
+ * [PaperDaily] section 二, third step: suitable projections run on low-bit
+ * weights and activations, with quantization fused next to the
+ * normalization.  Here: FP8 E4M3 (round to nearest even, saturating at 448)
+ * with one fp32 scale per row of each quantized operand -- per token for
+ * activations, per output channel for weights: s = amax / 448 (1 for an
+ * all-zero row), q = E4M3(value / s), amax, division and rounding in fp32.
+ * A projection computes (sum_k qa qw) * sa[row] * sw[col] + b on the tcgen05
+ * tensor cores (kind::f8f6f4, fp32 accumulation), then its epilogue. */
+
+/* Per-row E4M3 quantization of a [rows, cols] matrix `a` (device; fp32 or
+ * bf16 by `dtype`): q [rows, cols] E4M3 codes, s [rows] fp32 scales (device).
+ * cols % 16 == 0; a, q 16-byte aligned. */
+FSDIT_API fsdit_status fsdit_quantize_rows(const void* a, int dtype, int rows, int cols, uint8_t* q, float* s,
+                                           fsdit_stream_t stream);
+
+/* RMSNorm fused with the quantization of its output: y = x * rstd * g in
+ * fp32 (x fp32 [rows, hidden], g bf16), then q, s as fsdit_quantize_rows. */
+FSDIT_API fsdit_status fsdit_rmsnorm_quant(const float* x, const void* g, int rows, int hidden, float eps,
+                                           uint8_t* q, float* s, fsdit_stream_t stream);
+
+/* out = epilogue((qa qw^T) * sa[row] * sw[col] + b): qa [M, K], qw [N, K] E4M3
+ * codes, sa [M], sw [N] fp32, b bf16; epilogues and outputs as
+ * fsdit_linear with dtype bf16.  K % 16 == 0, N % 32 == 0, pointers 16-byte
+ * aligned. */
+FSDIT_API fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* qa, const float* sa, const uint8_t* qw,
+                                        const float* sw, const void* b, void* out, const float* resid,
+                                        const int32_t* pos, int M, int N, int K, int epilogue,
+                                        fsdit_stream_t stream);
 
 /* Joint attention ([tokendh] backbone section: one sequence of text,
  * video and audio tokens through one denoiser): for each head,

@@ -288,14 +288,16 @@ def broadcast_residual(x, y_c, keep_idx, near_idx, n_video):
 
 
 def dit_block_compressed(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video,
-                         rope_split=(32, 48, 48), eps=1e-6, theta=10000.0):
+                         rope_split=(32, 48, 48), eps=1e-6, theta=10000.0, block_fn=None):
     """The Flash compressed block, per-block form: gather, block, broadcast.
 
     RoPE positions of kept tokens are their original (t, h, w) coordinates
-    (Reading: the pages do not renumber them)."""
+    (Reading: the pages do not renumber them).  ``block_fn`` replaces
+    ``dit_block`` (e.g. the low-bit block of ``oracle.fp8``)."""
+    block_fn = block_fn or dit_block
     x_c = gather_rows(x, keep_idx, n_video)
     pos_c = gather_rows(pos, keep_idx, n_video)
-    y_c = dit_block(x_c, w, pos_c, heads, head_dim, rope_split, eps, theta)
+    y_c = block_fn(x_c, w, pos_c, heads, head_dim, rope_split, eps, theta)
     return broadcast_residual(x, y_c, keep_idx, near_idx, n_video)
 
 
@@ -388,7 +390,7 @@ def output_heads(x, io, modality, eps=1e-6):
 
 def dit_stack(layers, layer_compress, io, tok, time_table, video_lat, text_emb,
               audio_lat, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
-              theta=10000.0, segment=False):
+              theta=10000.0, segment=False, block_fn=None):
     """One backbone evaluation: embed, layers, heads -> (v_video, v_audio).
 
     ``tok`` holds the packed tags: ``modality``, ``time_id``, ``pos`` [n,3],
@@ -400,7 +402,11 @@ def dit_stack(layers, layer_compress, io, tok, time_table, video_lat, text_emb,
     before a run of compressed layers and broadcasts once after it; in exact
     arithmetic the two agree because kept rows only ever read kept rows and
     the dropped-row updates telescope.
+
+    ``block_fn`` replaces ``dit_block`` for every layer (e.g. the low-bit block
+    ``oracle.fp8.dit_block_fp8``); the default is the full-precision block.
     """
+    block_fn = block_fn or dit_block
     x = embed(io, tok["modality"], tok["time_id"], time_table, video_lat,
               text_emb, audio_lat)
     pos = tok["pos"]
@@ -408,18 +414,18 @@ def dit_stack(layers, layer_compress, io, tok, time_table, video_lat, text_emb,
     l = 0
     while l < L:
         if not layer_compress[l]:
-            x = dit_block(x, layers[l], pos, heads, head_dim, rope_split, eps, theta)
+            x = block_fn(x, layers[l], pos, heads, head_dim, rope_split, eps, theta)
             l += 1
         elif not segment:
             x = dit_block_compressed(x, layers[l], pos, heads, head_dim,
                                      tok["keep_idx"], tok["near_idx"], tok["n_video"],
-                                     rope_split, eps, theta)
+                                     rope_split, eps, theta, block_fn)
             l += 1
         else:
             x_c = gather_rows(x, tok["keep_idx"], tok["n_video"])
             pos_c = gather_rows(pos, tok["keep_idx"], tok["n_video"])
             while l < L and layer_compress[l]:
-                x_c = dit_block(x_c, layers[l], pos_c, heads, head_dim, rope_split,
+                x_c = block_fn(x_c, layers[l], pos_c, heads, head_dim, rope_split,
                                 eps, theta)
                 l += 1
             x = broadcast_residual(x, x_c, tok["keep_idx"], tok["near_idx"],
@@ -459,7 +465,7 @@ def euler_step(x, v, row_modality, out_mask, t_cur, t_next):
 
 def flow_sample(layers, layer_compress, io, tok, video_clock, audio_clock,
                 video_lat, text_emb, audio_lat, heads, head_dim,
-                rope_split=(32, 48, 48), eps=1e-6, theta=10000.0, segment=False):
+                rope_split=(32, 48, 48), eps=1e-6, theta=10000.0, segment=False, block_fn=None):
     """The few-step sampler: len(clock)-1 evaluations; evaluation e runs the
     stack with time table [0, t_v[e], t_a[e]] and moves target video rows from
     t_v[e] to t_v[e+1] and audio rows from t_a[e] to t_a[e+1].
@@ -473,7 +479,7 @@ def flow_sample(layers, layer_compress, io, tok, video_clock, audio_clock,
     for e in range(E):
         table = [0.0, video_clock[e], audio_clock[e]]
         v_vid, v_aud = dit_stack(layers, layer_compress, io, tok, table, vl, text_emb,
-                                 al, heads, head_dim, rope_split, eps, theta, segment)
+                                 al, heads, head_dim, rope_split, eps, theta, segment, block_fn)
         t_cur = [0.0, video_clock[e], audio_clock[e], 0.0]
         t_nxt = [0.0, video_clock[e + 1], audio_clock[e + 1], 0.0]
         vl = euler_step(vl, v_vid, tok["video_modality"], tok["video_out"], t_cur, t_nxt)
