@@ -119,12 +119,18 @@ def case_memory(a):
 
 def case_chunk(a):
     """One steady-state long-video chunk of the 42-layer Flash backbone: the
-    6x34x60 target (boundary + 5 future latents) plus a full 11-frame history
-    (4,140 rows), 3 evaluations, replayed from a CUDA graph."""
+    target grid (default 6x34x60: boundary + 5 future latents) plus a full
+    11-frame history (4,140 rows at 34x60), 3 evaluations, replayed from a
+    CUDA graph."""
     w = S.WORKLOADS["flash_backbone_6x34x60"]
+    if a.grid:
+        w = S.scaled(w, grid=tuple(int(v) for v in a.grid.split("x")))
     T, H, W = w.grid
     layers, io = S.make_weights(w, device="cuda")
-    bb = api.Backbone(api.dims_of(w), [api.BlockWeights(l) for l in layers], api.IOWeights(io), w.compress)
+    if a.fp8:
+        layers = [api.quantize_block_weights(l) for l in layers]
+    bb = api.Backbone(api.dims_of(w, proj_fp8=a.fp8), [api.BlockWeights(l) for l in layers], api.IOWeights(io),
+                      w.compress)
     inp = S.make_inputs(w, device="cuda")
     lv = api.LongVideo(bb, w.grid, w.n_text, w.n_audio, w.video_ch)
     g = torch.Generator(device="cuda").manual_seed(8)
@@ -161,7 +167,8 @@ def case_chunk(a):
 
     per_eval = sum(layer_flops(seq.n_compressed if c else tokens) for c in w.compress)
     tflop = per_eval * w.n_evals / 1e12
-    return {"case": "chunk", "tflop_per_chunk": tflop, "tflops": tflop / ms * 1e3, "workload": "flash_chunk_6x34x60_history11", "history_rows": rows, "tokens": tokens,
+    return {"case": "chunk", "tflop_per_chunk": tflop, "tflops": tflop / ms * 1e3, "fp8": bool(a.fp8),
+            "workload": f"flash_chunk_{T}x{H}x{W}_history11", "history_rows": rows, "tokens": tokens,
             "compressed_tokens": seq.n_compressed, "ms_per_chunk": ms,
             "tokens_per_s": tokens * w.n_evals / ms * 1e3, "new_frames_per_s": 17 / ms * 1e3,
             "gather_ms": g_ms, "gather_gbs": rows * (w.video_ch * 8 + 12) / g_ms / 1e6}
@@ -177,7 +184,8 @@ def main():
     p.add_argument("--K", type=int, default=5376)
     p.add_argument("--epi", default="qkv", choices=sorted(EPI))
     p.add_argument("--workload", default="flash_block_6x34x60")
-    p.add_argument("--fp8", action="store_true", help="gemm: E4M3 operands (per-row scales)")
+    p.add_argument("--fp8", action="store_true", help="gemm / chunk: E4M3 projections (per-row scales)")
+    p.add_argument("--grid", default="", help="chunk: target latent grid TxHxW (default 6x34x60)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
