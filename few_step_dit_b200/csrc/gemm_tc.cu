@@ -191,9 +191,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // Pair-tile variant: a cluster of two CTAs computes a 256 x 256 output tile
 // with tcgen05.mma.cta_group::2.  Each CTA stages only its own 128 A rows and
-// 128 of the 256 B rows per K step (32 KB a stage instead of 48 KB for the
-// same 128 x 256 share of the output), which halves the B operand's
-// shared-memory and L2 traffic per FLOP.  Roles per CTA as above; warp 1 of
+// 128 of the 256 B rows per K step, which halves the B operand's
+// shared-memory and L2 traffic per FLOP.  A stage holds two 128-byte-wide
+// boxes of each operand (64 KB per CTA, 3 stages): eight MMAs per barrier
+// round trip.  Roles per CTA as above; warp 1 of
 // CTA rank 0 issues the pair MMAs.  Both CTAs' TMA copies of a stage complete
 // on rank 0's `full` barrier (rank 0 expects the bytes of both); the MMA
 // commits release the stage in both CTAs.  Accumulator rows 0..127 of a tile
@@ -205,9 +206,10 @@ namespace gemm2 {
 constexpr int BM = 256, BN = 256, BK = 64;  // BK: bf16 elements per stage row (128 bytes)
 constexpr int BK8 = 128;                     // E4M3 elements per stage row (128 bytes)
 constexpr int HM = BM / 2, HN = BN / 2;  // per-CTA share of A rows and B rows
-constexpr int STAGES = 6;
-constexpr int A_BYTES = HM * BK * 2;
-constexpr int B_BYTES = HN * BK * 2;
+constexpr int STAGES = 3;
+constexpr int BOXES = 2;  // 128-byte boxes per operand per stage
+constexpr int A_BYTES = HM * BK * 2 * BOXES;
+constexpr int B_BYTES = HN * BK * 2 * BOXES;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each on half the columns
@@ -226,7 +228,8 @@ template <bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const gemm::Args args) {
-  constexpr int BKE = FP8 ? BK8 : BK;  // K elements per stage
+  constexpr int BKE = (FP8 ? BK8 : BK) * BOXES;  // K elements per stage
+  constexpr int BOXE = FP8 ? BK8 : BK;          // K elements per box
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -290,8 +293,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sa = base + s * STAGE_BYTES;
           const uint32_t full = full0 + 8u * (uint32_t)s;
           if (rank == 0) mbar_expect_tx(FULL(s), 2 * STAGE_BYTES);
-          tma_load_2d_pair(sa, &tmA, kb * BKE, row_a, full);
-          tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BKE, row_b, full);
+          for (int bx = 0; bx < BOXES; ++bx) {
+            tma_load_2d_pair(sa + bx * (HM * 128), &tmA, kb * BKE + bx * BOXE, row_a, full);
+            tma_load_2d_pair(sa + A_BYTES + bx * (HN * 128), &tmB, kb * BKE + bx * BOXE, row_b, full);
+          }
           last_s = s;
           last_ph = ph;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -322,14 +327,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(FULL(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + A_BYTES;
-          // four MMAs of 32 bytes of K each (16 bf16 or 32 E4M3 elements)
+          // eight MMAs of 32 bytes of K each (16 bf16 or 32 E4M3 elements), four per box
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 4 * BOXES; ++k) {
+            const uint32_t oa = (uint32_t)((k >> 2) * (HM * 128) + (k & 3) * 32);
+            const uint32_t ob = (uint32_t)((k >> 2) * (HN * 128) + (k & 3) * 32);
             if constexpr (FP8)
-              mma_e4m3_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC_FP8,
+              mma_e4m3_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC_FP8,
                                (kb | k) != 0 ? 1u : 0u);
             else
-              mma_bf16_ss_pair(d, sw128_desc(sa + 32 * k, 16, 1024), sw128_desc(sb + 32 * k, 16, 1024), IDESC,
+              mma_bf16_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC,
                                (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit_pair(EMPTY(s));
