@@ -75,11 +75,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def gemm_sources_sha256():
+def _code_lines(text):
+    """Source text without // comments and blank lines: the hash follows code changes only."""
+    out = []
+    for line in text.splitlines():
+        line = line.split("//", 1)[0].rstrip()
+        if line.strip():
+            out.append(line)
+    return "\n".join(out)
+
+
+def gemm_sources_sha256(read=None):
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(rel)
+        h.update(_code_lines(text).encode())
     return h.hexdigest()
 
 

@@ -2,7 +2,7 @@
 //
 // One CTA per SM (grid = min(tiles, SMs)), 192 threads in three roles:
 //   warp 0  lane 0: TMA producer -- 128x64 A and 256x64 B tiles (128-byte
-//           swizzle, no multicast) into a 4-stage shared-memory ring;
+//           swizzle; each CTA loads only for itself) into a 4-stage ring;
 //   warp 1  allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //           (128x256x16, fp32 accumulators in TMEM, double-buffered) and
 //           tcgen05.commit to release ring stages / publish accumulators;

@@ -1,5 +1,5 @@
 // Inline-PTX wrappers for sm_100a: mbarriers (with bounded waits), TMA tile
-// loads (no multicast), tensor-memory allocation, tcgen05.mma / commit / ld /
+// loads (each into the issuing CTA only), tensor-memory allocation, tcgen05.mma / commit / ld /
 // st and shared-memory matrix descriptors.
 #pragma once
 
@@ -247,7 +247,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 }
 // 2D tiled load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (`cluster_bar`, a shared::cluster
-// address); no multicast.
+// address); the copy lands in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* tm, int c0, int c1,
                                                  uint32_t cluster_bar) {
   asm volatile(
