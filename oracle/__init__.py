@@ -17,11 +17,15 @@ Sources (web write-ups of arXiv 2609.15863, "LynnReal-Omni"):
   section 二 "Flash怎么把22帧压到377毫秒" (compression, residual broadcast),
   section 三 "长视频不是无限塞历史，而是保留“够用的记忆”" (chunked long video).
 * [tokendh] section "长视频生成：怎么记住十分钟前发生的事" (boundary frame,
-  bounded multi-stride history).
+  bounded multi-stride history) and section "解码器瓶颈：被忽视的那一半时间"
+  (the 26-layer lightweight decoder).
+* [ananclaw explainer] papers.ananclaw.com explainer of 2609.15863, section 3.4
+  "推理加速" (the Flash model's lightweight VAE decoder).
 
 Modules: ``dit.py`` (block, compression, stack, flow-matching sampler),
 ``long_video.py`` (chunked generation with the bounded history; import it as
-``oracle.long_video``) and ``fp8.py`` (E4M3 block projections; ``oracle.fp8``).
+``oracle.long_video``), ``fp8.py`` (E4M3 block projections; ``oracle.fp8``)
+and ``decoder.py`` (the lightweight decoder's forward; ``oracle.decoder``).
 
 Every floating-point step runs in float64.  Where the pages leave a step open
 the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
@@ -29,7 +33,8 @@ the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
 Parity status per function: everything in ``dit.py`` is pinned by the CPU
 tests in ``tests/test_oracle_pins.py`` and everything in ``long_video.py`` by
 ``tests/test_oracle_long_video.py``, everything in ``fp8.py`` by
-``tests/test_oracle_fp8.py``, except the conventions that are pure
+``tests/test_oracle_fp8.py`` and everything in ``decoder.py`` by
+``tests/test_oracle_decoder.py``, except the conventions that are pure
 definitions (weight init, time-embedding MLP, bias placement); those are
 "parity unpinned" in the sense that no page fixes them, so the GPU path is
 compared against this oracle's definition of them.
