@@ -407,3 +407,48 @@ class LongVideo:
         self.bb.sample(seq, video_clock, audio_clock, vl, text_emb, al, stream=stream)
         self.store.push(vl[hw:n_grid] if has_b else vl[:n_grid], stream)
         return vl[:n_grid], al
+
+
+# ---------------------------------------------------------------- decoder
+
+class DecoderIO:
+    """Latent projection, final RMSNorm gain and pixel head of the decoder
+    (w_in [hidden, c_lat], b_in, g_out, w_out [c_pix*patch_t*patch_s^2, hidden], b_out)."""
+
+    def __init__(self, tensors: dict, c_pix=3, patch_t=4, patch_s=16):
+        self.tensors = {k: v.contiguous() for k, v in tensors.items()}
+        t = self.tensors
+        if t["w_out"].shape[0] != c_pix * patch_t * patch_s * patch_s:
+            raise ValueError("w_out must have c_pix * patch_t * patch_s^2 rows")
+        self.struct = L.DecoderIO(*[t[k].data_ptr() for k in L.DECODER_IO_FIELDS], t["w_in"].shape[1],
+                                  c_pix, patch_t, patch_s)
+
+
+class Decoder:
+    """The lightweight video decoder: latents [T*H*W, c_lat] (cells (t, h, w)
+    row-major) -> pixels [1 + patch_t*(T-1), c_pix, H*patch_s, W*patch_s]."""
+
+    def __init__(self, dims, layers, io: DecoderIO):
+        self.dims = dims
+        self.layers = layers
+        self.io = io
+        self.n_layers = len(layers)
+        self.layer_structs = (L.BlockWeights * max(self.n_layers, 1))(*[lw.struct for lw in layers])
+
+    def frames(self, T):
+        return L.load().fsdit_decoder_frames(T, self.io.struct.patch_t)
+
+    def workspace_bytes(self, grid):
+        T, H, W = grid
+        return L.load().fsdit_decoder_workspace_size(C.byref(self.dims), C.byref(self.io.struct), T, H, W)
+
+    def forward(self, latents, grid, pixels=None, stream=None):
+        T, H, W = grid
+        s = self.io.struct
+        if pixels is None:
+            pixels = torch.empty(self.frames(T), s.c_pix, H * s.patch_s, W * s.patch_s, dtype=torch.float32,
+                                 device=latents.device)
+        ws = workspace(self.workspace_bytes(grid), latents.device)
+        L.call("fsdit_decoder_forward", C.byref(self.dims), self.n_layers, self.layer_structs, C.byref(s), T, H, W,
+               L.ptr(latents), L.ptr(pixels), L.ptr(ws), ws.numel(), _stream(stream))
+        return pixels

@@ -17,7 +17,7 @@ static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "ge
                                            "broadcast",     "embed",         "time_mlp",  "heads",
                                            "euler",         "keep_map",  "rope_table", "history_gather",
                                            "quantize",      "gemm_fp8_qkv_rope", "gemm_fp8_residual",
-                                           "gemm_fp8_gelu"};
+                                           "gemm_fp8_gelu", "grid_positions", "pixel_head"};
 struct Prof {
   bool on = false;
   int used = 0;
@@ -172,15 +172,18 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.log2_theta = log2f(d->rope_theta);
   e.row_scale = nullptr;
   e.col_scale = nullptr;
+  e.up_h = e.up_w = e.up_c = e.up_pt = e.up_ps = 1;
   return e;
 }
 
 fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, const EpiParams& ep, int M, int N,
                            int K, cudaStream_t st, int prof_cls) {
   if (M <= 0) return FSDIT_OK;
-  static const int cls_of[5] = {PC_GEMM_BIAS, PC_GEMM_BIAS_F32, PC_GEMM_QKV, PC_GEMM_GELU, PC_GEMM_RESID};
+  static const int cls_of[6] = {PC_GEMM_BIAS, PC_GEMM_BIAS_F32, PC_GEMM_QKV, PC_GEMM_GELU, PC_GEMM_RESID,
+                                PC_PIXEL_HEAD};
   const double s = (double)dsize(d->dtype);
-  const double out_b = (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32) ? 4.0 : s;
+  const double out_b =
+      (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32 || ep.epi == EPI_UNPATCH) ? 4.0 : s;
   const double by = ((double)M * K + (double)N * K) * s + (double)M * N * out_b +
                     (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
   ProfScope ps(prof_cls >= 0 ? prof_cls : cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);

@@ -68,7 +68,30 @@ struct EpiParams {
   float log2_theta;
   const float* row_scale;  // [M] or null: accumulators are multiplied by
   const float* col_scale;  // row_scale[row] * col_scale[col] (FP8 dequantization) before the bias
+  int up_h, up_w;          // EPI_UNPATCH: the rows are the cells of a (t, h, w) grid up_h x up_w per frame,
+  int up_c, up_pt, up_ps;  // each column a pixel of the cell's up_c x up_pt x up_ps x up_ps patch
 };
+
+// Decoder pixel head (internal epilogue, not reachable through fsdit_linear):
+// out (f32) = acc + b written straight into frames [F][up_c][up_h*ps][up_w*ps].
+// Column (c, dt, dy, dx) of cell (t, h, w), dx fastest, is frame
+// pt*t + dt - (pt - 1) (dropped when negative: latent frame 0 yields one
+// frame), pixel (ps*h + dy, ps*w + dx).
+constexpr int EPI_UNPATCH = 5;
+
+// Element offset of column `col` of row `row` in the frames, -1 if dropped.
+__device__ __forceinline__ long long unpatch_offset(const EpiParams& p, int row, int col) {
+  const int ps = p.up_ps, pt = p.up_pt;
+  const int dx = col % ps, r1 = col / ps;
+  const int dy = r1 % ps, r2 = r1 / ps;
+  const int dt = r2 % pt, ch = r2 / pt;
+  const int w = row % p.up_w, r = row / p.up_w;
+  const int h = r % p.up_h, t = r / p.up_h;
+  const int f = t * pt + dt - (pt - 1);
+  if (f < 0) return -1;
+  const long long hp = (long long)p.up_h * ps, wp = (long long)p.up_w * ps;
+  return (((long long)f * p.up_c + ch) * hp + (long long)h * ps + dy) * wp + (long long)w * ps + dx;
+}
 
 // Apply the epilogue to `cnt` consecutive columns [col, col+cnt) of one row.
 // v[] holds the fp32 accumulators; cnt is even and col is even.
@@ -107,7 +130,14 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
 #pragma unroll
     for (int i = 0; i < CNT; ++i) v[i] = gelu_tanh(v[i]);
   }
-  if (p.epi == FSDIT_EPI_RESIDUAL) {
+  if (p.epi == EPI_UNPATCH) {
+    float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+    for (int i = 0; i < CNT; ++i) {
+      const long long off = unpatch_offset(p, row, col + i);
+      if (off >= 0) o[off] = v[i];
+    }
+  } else if (p.epi == FSDIT_EPI_RESIDUAL) {
     const float* r = p.resid + (size_t)row * p.ldr + col;
     float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
     if constexpr (CNT % 4 == 0) {
@@ -248,7 +278,17 @@ __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_bf16out(v[i]);
   }
-  if (p.epi == FSDIT_EPI_RESIDUAL) {
+  if (p.epi == EPI_UNPATCH) {
+    // up_ps % 4 == 0: each group of 4 columns is 4 adjacent pixels of one
+    // pixel row, 16-byte aligned in the frames
+    float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const long long off = unpatch_offset(p, row, col + 4 * i);
+      if (off >= 0)
+        *reinterpret_cast<float4*>(o + off) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  } else if (p.epi == FSDIT_EPI_RESIDUAL) {
     float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -284,7 +324,7 @@ namespace fsdit {
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
   PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_QUANT,
-  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_COUNT
+  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_GRID_POS, PC_PIXEL_HEAD, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);

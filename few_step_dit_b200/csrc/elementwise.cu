@@ -181,7 +181,8 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int rows, int
 // ---------------------------------------------------------------- embedding
 // x[r] = src(r) + mod_emb[modality[r]] + temb[time_id[r]], where src(r) is the
 // small-K projection lat[r'] W^T + b of a video/control or audio row, or the
-// precomputed text projection row.  A block owns EMB_RB rows of one segment
+// precomputed text projection row.  Without tags (modality == nullptr: the
+// decoder's latent cells) x[r] = src(r).  A block owns EMB_RB rows of one segment
 // and EMB_CB consecutive columns: each thread keeps its column's weight row
 // in registers; the rows' latents, modality and timestep embeddings of the
 // block's columns are staged in shared memory; stores are coalesced.
@@ -202,7 +203,8 @@ __global__ void __launch_bounds__(256) embed_kernel(
   const int nr = min(EMB_RB, rows - rb0);
   const int c = blockIdx.y * EMB_CB + threadIdx.x;
   const bool col_ok = c < hidden;
-  if (threadIdx.x < EMB_RB) {
+  const bool tagged = modality != nullptr;
+  if (tagged && threadIdx.x < EMB_RB) {
     int m = expect_a, t = 0;
     if (threadIdx.x < nr) {
       const int r = row0 + rb0 + threadIdx.x;
@@ -223,9 +225,11 @@ __global__ void __launch_bounds__(256) embed_kernel(
       s_lat[rr][kk] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
     }
   }
+  if (tagged) {
 #pragma unroll
-  for (int m = 0; m < 4; ++m) s_mod[m][threadIdx.x] = col_ok ? ld_f32<TW>(mod_emb + (size_t)m * hidden + c) : 0.f;
-  for (int t = 0; t < n_times; ++t) s_temb[t][threadIdx.x] = col_ok ? temb[(size_t)t * hidden + c] : 0.f;
+    for (int m = 0; m < 4; ++m) s_mod[m][threadIdx.x] = col_ok ? ld_f32<TW>(mod_emb + (size_t)m * hidden + c) : 0.f;
+    for (int t = 0; t < n_times; ++t) s_temb[t][threadIdx.x] = col_ok ? temb[(size_t)t * hidden + c] : 0.f;
+  }
   __syncthreads();
   if (!col_ok) return;
   float wr[KMAX];
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(256) embed_kernel(
     } else {
       acc = text_proj[(size_t)(rb0 + j) * hidden + c];
     }
-    acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
+    if (tagged) acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
     x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
   }
 }

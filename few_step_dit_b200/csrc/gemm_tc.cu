@@ -545,8 +545,9 @@ fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep,
   // pair tiles once there are two 128-row blocks to share them; their
   // epilogue moves bias, output, residual and RoPE table in 16-byte pieces
   auto a16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  const bool f32_out = ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32;
+  const bool f32_out = ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32 || ep.epi == EPI_UNPATCH;
   const bool vec_ok = a16(ep.bias) && a16(ep.out) && ep.ldo % (f32_out ? 4 : 8) == 0 &&
+                      (ep.epi != EPI_UNPATCH || ep.up_ps % 4 == 0) &&
                       (ep.epi != FSDIT_EPI_RESIDUAL || (a16(ep.resid) && ep.ldr % 4 == 0)) &&
                       (ep.rope_cs == nullptr || a16(ep.rope_cs)) && (ep.head_dim & (ep.head_dim - 1)) == 0;
   if (M > gemm2::HM && vec_ok) {

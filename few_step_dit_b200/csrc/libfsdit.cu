@@ -8,3 +8,4 @@
 #include "attn_tc.cu"
 #include "noalloc.cu"
 #include "history.cu"
+#include "decoder.cu"

@@ -4,6 +4,8 @@ Examples:
   python -m few_step_dit_b200.kernel_bench attention --n 12560 --heads 56
   python -m few_step_dit_b200.kernel_bench gemm --M 12560 --N 21504 --K 5376 --epi qkv
   python -m few_step_dit_b200.kernel_bench block --workload flash_block_6x34x60
+  python -m few_step_dit_b200.kernel_bench decoder [--grid 6x34x60] [--fp8]
+  python -m few_step_dit_b200.kernel_bench generate   # 3-eval Flash pass + decoder
 Inputs are seeded Gaussians; each case prints one JSON line.
 """
 
@@ -174,9 +176,96 @@ def case_chunk(a):
             "gather_ms": g_ms, "gather_gbs": rows * (w.video_ch * 8 + 12) / g_ms / 1e6}
 
 
+def _decoder(a, device="cuda"):
+    w = S.DECODER_WORKLOADS["decoder_6x34x60"]
+    if a.grid:
+        w = S.scaled(w, grid=tuple(int(v) for v in a.grid.split("x")))
+    layers, io = S.make_decoder_weights(w, device=device)
+    if a.fp8:
+        layers = [api.quantize_block_weights(l) for l in layers]
+    dec = api.Decoder(api.dims_of(w, proj_fp8=a.fp8), [api.BlockWeights(l) for l in layers],
+                      api.DecoderIO(io, w.c_pix, w.patch_t, w.patch_s))
+    return w, dec
+
+
+def _decoder_flops(w):
+    n, A, Hd, F = w.n_cells, w.attn_dim, w.hidden, w.ffn
+    per_layer = 2.0 * n * (4 * A * Hd + 2 * Hd * F) + 4.0 * n * n * A
+    return w.n_layers * per_layer + 2.0 * n * Hd * (w.c_lat + w.pixel_cols)
+
+
+def _graph_ms(step, a):
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    ms = time_it(graph.replay, a.iters, a.warmup)
+    del graph
+    return ms
+
+
+def _profile(step):
+    step()
+    torch.cuda.synchronize()
+    L.profile_start()
+    step()
+    prof = L.profile_stop()
+    tot = sum(v["ms"] for v in prof.values())
+    return {k: {"ms": round(v["ms"], 3), "share": round(v["ms"] / tot, 4),
+                "tflops": round(v["flops"] / v["ms"] / 1e9, 1) if v["flops"] else None,
+                "gbs": round(v["bytes"] / v["ms"] / 1e6, 1)} for k, v in prof.items()}
+
+
+def case_decoder(a):
+    """The 26-layer lightweight decoder (hidden 2048, 16 heads, FFN 8192) on
+    a latent grid (default 6x34x60 -> 21 frames of 544x960), replayed from a
+    CUDA graph; plus a per-kernel-class profile of one eager run."""
+    w, dec = _decoder(a)
+    lat = S.make_decoder_latents(w, device="cuda")
+    px = torch.empty(w.pixel_shape, device="cuda")
+    step = lambda: dec.forward(lat, w.grid, pixels=px)  # noqa: E731
+    ms = _graph_ms(step, a)
+    tflop = _decoder_flops(w) / 1e12
+    T, H, W = w.grid
+    return {"case": "decoder", "workload": f"decoder_{T}x{H}x{W}", "fp8": bool(a.fp8), "cells": w.n_cells,
+            "frames": w.n_frames, "ms": ms, "tflop": tflop, "tflops": tflop / ms * 1e3,
+            "frames_per_s": w.n_frames / ms * 1e3, "classes": _profile(step)}
+
+
+def case_generate(a):
+    """The pages' latency protocol on one GPU: the 3-evaluation Flash
+    backbone pass (42 layers, 6x34x60, text 256, audio 64) followed by the
+    26-layer decoder of its video latents, one CUDA graph, warm."""
+    wb = S.WORKLOADS["flash_backbone_6x34x60"]
+    layers, io = S.make_weights(wb, device="cuda")
+    if a.fp8:
+        layers = [api.quantize_block_weights(l) for l in layers]
+    bb = api.Backbone(api.dims_of(wb, proj_fp8=a.fp8), [api.BlockWeights(l) for l in layers], api.IOWeights(io),
+                      wb.compress)
+    seq = api.Sequence.from_workload(wb, S.pack_tokens(wb), "cuda")
+    inp = S.make_inputs(wb, device="cuda")
+    wd, dec = _decoder(a)
+    assert wd.grid == wb.grid and wd.c_lat == wb.video_ch
+    vl, al = inp["video_lat"].clone(), inp["audio_lat"].clone()
+    px = torch.empty(wd.pixel_shape, device="cuda")
+
+    def step():
+        vl.copy_(inp["video_lat"])
+        al.copy_(inp["audio_lat"])
+        bb.sample(seq, wb.video_clock, wb.audio_clock, vl, inp["text_emb"], al)
+        dec.forward(vl, wd.grid, pixels=px)
+
+    ms = _graph_ms(step, a)
+    ms_dec = _graph_ms(lambda: dec.forward(vl, wd.grid, pixels=px), a)
+    return {"case": "generate", "workload": "flash_backbone_6x34x60+decoder_6x34x60", "fp8": bool(a.fp8),
+            "ms": ms, "ms_decoder": ms_dec, "ms_backbone": ms - ms_dec, "frames": wd.n_frames,
+            "frames_per_s": wd.n_frames / ms * 1e3}
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk"])
+    p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk", "decoder", "generate"])
     p.add_argument("--n", type=int, default=12560)
     p.add_argument("--heads", type=int, default=56)
     p.add_argument("--M", type=int, default=12560)
@@ -184,15 +273,17 @@ def main():
     p.add_argument("--K", type=int, default=5376)
     p.add_argument("--epi", default="qkv", choices=sorted(EPI))
     p.add_argument("--workload", default="flash_block_6x34x60")
-    p.add_argument("--fp8", action="store_true", help="gemm / chunk: E4M3 projections (per-row scales)")
-    p.add_argument("--grid", default="", help="chunk: target latent grid TxHxW (default 6x34x60)")
+    p.add_argument("--fp8", action="store_true",
+                   help="gemm / chunk / decoder / generate: E4M3 projections (per-row scales)")
+    p.add_argument("--grid", default="", help="chunk / decoder: latent grid TxHxW (default 6x34x60)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
     B.build()
     L.load()
     res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
-           "memory": case_memory, "chunk": case_chunk}[a.case](a)
+           "memory": case_memory, "chunk": case_chunk, "decoder": case_decoder,
+           "generate": case_generate}[a.case](a)
     api.device_error()
     print(json.dumps(res), flush=True)
 

@@ -70,6 +70,13 @@ class HistoryStore(C.Structure):
 HISTORY_MAX_ENTRIES = 11
 HISTORY_MIN_SLOTS = 12
 
+DECODER_IO_FIELDS = ("w_in", "b_in", "g_out", "w_out", "b_out")
+
+
+class DecoderIO(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in DECODER_IO_FIELDS] + [
+        ("c_lat", C.c_int), ("c_pix", C.c_int), ("patch_t", C.c_int), ("patch_s", C.c_int)]
+
 
 class ProfEntry(C.Structure):
     _fields_ = [("name", C.c_char * 32), ("scopes", C.c_int), ("launches", C.c_int),
@@ -117,6 +124,10 @@ _SIGS = {
     "fsdit_history_gather": (_I, [C.POINTER(HistoryStore), C.POINTER(HistoryEntry), _I, _P, _I, _P, _P]),
     "fsdit_history_copy_frame": (_I, [C.POINTER(HistoryStore), _I, _P, _P]),
     "fsdit_chunk_tags": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "fsdit_decoder_frames": (_I, [_I, _I]),
+    "fsdit_decoder_workspace_size": (C.c_size_t, [C.POINTER(Dims), C.POINTER(DecoderIO), _I, _I, _I]),
+    "fsdit_decoder_forward": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(DecoderIO), _I, _I,
+                                   _I, _P, _P, _P, C.c_size_t, _P]),
 }
 
 _lib = None

@@ -115,6 +115,63 @@ WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class DecoderWorkload:
+    """Shapes of the lightweight video decoder: a transformer over the latent
+    cells of a T x H x W grid (hidden 2048, 26 layers, FFN 4 x hidden), each
+    cell decoded to a c_pix x patch_t x patch_s x patch_s pixel patch."""
+    name: str
+    hidden: int = 2048
+    heads: int = 16
+    head_dim: int = 128
+    ffn: int = 8192
+    n_layers: int = 26
+    grid: tuple = (6, 34, 60)
+    c_lat: int = 24
+    c_pix: int = 3
+    patch_t: int = 4
+    patch_s: int = 16
+    dtype: str = "bf16"
+    rope_split: tuple = (32, 48, 48)
+    rms_eps: float = 1e-6
+    rope_theta: float = 10000.0
+
+    @property
+    def attn_dim(self):
+        return self.heads * self.head_dim
+
+    @property
+    def n_cells(self):
+        T, H, W = self.grid
+        return T * H * W
+
+    @property
+    def n_frames(self):
+        return 1 + self.patch_t * (self.grid[0] - 1)
+
+    @property
+    def pixel_cols(self):
+        return self.c_pix * self.patch_t * self.patch_s * self.patch_s
+
+    @property
+    def pixel_shape(self):
+        T, H, W = self.grid
+        return (self.n_frames, self.c_pix, H * self.patch_s, W * self.patch_s)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+DECODER_WORKLOADS = {
+    # tiny fp32 decoder, checkable on the CPU in seconds
+    "tiny_decoder_f32": DecoderWorkload("tiny_decoder_f32", hidden=256, heads=2, ffn=1024, n_layers=2,
+                                        grid=(3, 4, 5), patch_s=4, dtype="f32"),
+    # the 26-layer decoder on the 540p clip's 6 x 34 x 60 latents -> 21 x 3 x 544 x 960
+    "decoder_6x34x60": DecoderWorkload("decoder_6x34x60"),
+}
+
+
 def scaled(w: Workload, **kw) -> Workload:
     """A copy of a workload with some fields replaced (smaller test cases)."""
     return replace(w, **kw)
@@ -260,3 +317,26 @@ def to_numpy64(d):
         else:
             out[k] = v
     return out
+
+
+def make_decoder_weights(w: DecoderWorkload, device="cpu", seed=SEED_WEIGHTS, n_layers=None):
+    """Decoder weights: (list of block weights, io dict with w_in [hidden,
+    c_lat], b_in, g_out, w_out [pixel_cols, hidden], b_out); same init recipe
+    as the backbone's."""
+    g = _gen(seed, device)
+    L = w.n_layers if n_layers is None else n_layers
+    layers = [make_block_weights(w, g, device) for _ in range(L)]
+    dt, H, s = w.torch_dtype, w.hidden, 0.02
+    io = {
+        "w_in": _randn((H, w.c_lat), g, s, dt, device),
+        "b_in": _randn((H,), g, s, dt, device),
+        "w_out": _randn((w.pixel_cols, H), g, s, dt, device),
+        "b_out": _randn((w.pixel_cols,), g, s, dt, device),
+    }
+    io["g_out"] = (1.0 + _randn((H,), g, s, torch.float32, device)).to(dt)
+    return layers, io
+
+
+def make_decoder_latents(w: DecoderWorkload, device="cpu", seed=SEED_INPUTS):
+    """Latents [T*H*W, c_lat] fp32, N(0, 1), cells (t, h, w) row-major."""
+    return _randn((w.n_cells, w.c_lat), _gen(seed, device), 1.0, torch.float32, device)

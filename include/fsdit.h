@@ -440,6 +440,55 @@ FSDIT_API fsdit_status fsdit_chunk_tags(int T, int H, int W, int base, int has_b
                                         int n_audio, uint8_t* modality, uint8_t* time_id, uint8_t* out_mask,
                                         int32_t* pos);
 
+/* ------------------------------------------------------------------ decoder
+ * The lightweight video decoder ([tokendh] section "解码器瓶颈：被忽视的那一半
+ * 时间": 26 layers, hidden width 2048, feed-forward 4x hidden; [ananclaw
+ * explainer] section 3.4: a lightweight VAE decoder), read as a transformer
+ * over the latent cells of a T x H x W grid:
+ *   x = z W_in^T + b_in  (one row per cell, (t, h, w) row-major; no time or
+ *                         modality embedding);
+ *   n_layers blocks of the backbone's form (fsdit_block_weights; RoPE at the
+ *   cell's (t, h, w); full attention over the clip; never compressed);
+ *   pixel head: rmsnorm(x; g_out) W_out^T + b_out, one row of
+ *   c_pix * patch_t * patch_s^2 values per cell, columns ordered
+ *   (channel, dt, dy, dx) with dx fastest;
+ *   unpatchify (fused into the head's epilogue): column (c, dt, dy, dx) of
+ *   cell (t, h, w) is pixel (patch_s*h + dy, patch_s*w + dx) of channel c in
+ *   frame patch_t*t + dt - (patch_t - 1), dropped when negative (causal:
+ *   latent frame 0 yields one frame), so T latent frames give
+ *   fsdit_decoder_frames(T, patch_t) = 1 + patch_t*(T - 1) frames. */
+typedef struct {
+  const void *w_in, *b_in;   /* [hidden, c_lat], [hidden] (dims.dtype, device) */
+  const void* g_out;         /* [hidden] final RMSNorm gain */
+  const void *w_out, *b_out; /* [c_pix*patch_t*patch_s*patch_s, hidden], [same] */
+  int c_lat;                 /* latent channels, 1..64 */
+  int c_pix;                 /* pixel channels (3) */
+  int patch_t;               /* frames per latent frame (4) */
+  int patch_s;               /* pixels per latent cell along h and w (16); a multiple of 4 */
+} fsdit_decoder_io;
+
+/* Frames decoded from T latent frames: 1 + patch_t*(T-1) (0 when T <= 0). */
+FSDIT_API int fsdit_decoder_frames(int T, int patch_t);
+
+/* Workspace bytes of fsdit_decoder_forward on a T x H x W grid (0 on bad
+ * arguments). */
+FSDIT_API size_t fsdit_decoder_workspace_size(const fsdit_dims* dims, const fsdit_decoder_io* io, int T, int H,
+                                              int W);
+
+/* Decode latents (device, fp32 [T*H*W][c_lat], cells (t, h, w) row-major) into
+ * pixels (device, fp32 [fsdit_decoder_frames(T, patch_t)][c_pix][H*patch_s]
+ * [W*patch_s], 16-byte aligned, fully written).  layers: host array of
+ * n_layers block weights (device pointers; with dims.proj_fp8 the E4M3 weights
+ * and scales as for the backbone).  The residual stream is fp32; the GEMMs and
+ * attention run as in the backbone (bf16 on the tcgen05 tensor cores, or
+ * exact fp32 with dims.dtype FSDIT_F32).  Errors: FSDIT_E_NULL,
+ * FSDIT_E_SHAPE (grid empty, c_lat outside 1..64, patch sizes not positive,
+ * patch_s % 4 != 0), FSDIT_E_ALIGN, FSDIT_E_WORKSPACE. */
+FSDIT_API fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
+                                             const fsdit_decoder_io* io, int T, int H, int W, const float* latents,
+                                             float* pixels, void* workspace, size_t ws_bytes,
+                                             fsdit_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -96,3 +96,44 @@ def test_block_forward_rejects_inconsistent_tokens(fs):
     tok.n_keep = 30
     # workspace too small
     assert fs.dit_block_forward(C.byref(d), C.byref(w), C.byref(tok), fake, fake, fake, 16, None) == -6
+
+
+def _dec_io(**kw):
+    io = L.DecoderIO(*([0x10000] * 5), 24, 3, 4, 16)
+    for k, v in kw.items():
+        setattr(io, k, v)
+    return io
+
+
+def test_decoder_frame_count_closed_form(fs):
+    assert fs.fsdit_decoder_frames(6, 4) == 21
+    assert fs.fsdit_decoder_frames(1, 4) == 1
+    assert fs.fsdit_decoder_frames(5, 4) == 17
+    assert fs.fsdit_decoder_frames(0, 4) == 0
+
+
+def test_decoder_workspace_size_and_bad_io(fs):
+    d = api.make_dims(2048, 16, 8192, L.BF16)
+    n = fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io()), 6, 34, 60)
+    # fp32 residual + bf16 GEMM operands (x_n, qkv, FFN) for 12,240 cells
+    assert n >= 12240 * (2048 * 4 + (2048 + 3 * 2048 + 8192) * 2)
+    assert fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io(patch_s=6)), 6, 34, 60) == 0
+    assert fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io(c_lat=0)), 6, 34, 60) == 0
+    assert fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io(c_lat=65)), 6, 34, 60) == 0
+    assert fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io()), 0, 34, 60) == 0
+    assert fs.fsdit_decoder_workspace_size(C.byref(d), C.byref(_dec_io(w_out=None)), 6, 34, 60) == 0
+
+
+def test_decoder_forward_rejects_bad_arguments_without_launching(fs):
+    d = api.make_dims(2048, 16, 8192, L.BF16)
+    fake, odd = C.c_void_p(0x10000), C.c_void_p(0x10004)
+    w = (L.BlockWeights * 1)(L.BlockWeights(*([0x10000] * 10)))
+    big = 1 << 40
+    f = fs.fsdit_decoder_forward
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, None, fake, fake, big, None) == -1
+    assert f(C.byref(d), 1, None, C.byref(_dec_io()), 6, 34, 60, fake, fake, fake, big, None) == -1
+    assert f(C.byref(d), 1, w, C.byref(_dec_io(patch_s=2)), 6, 34, 60, fake, fake, fake, big, None) == -2
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 0, 60, fake, fake, fake, big, None) == -2
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, odd, fake, big, None) == -3
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, fake, fake, 1024, None) == -6
+    assert "workspace" in L.last_error()

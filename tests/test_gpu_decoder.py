@@ -1,0 +1,160 @@
+"""The decoder's forward pass on the GPU against the oracle.
+
+* fp32 (exact FMA GEMMs, fp32 attention): rel-L2 <= 1e-5 on every pixel, with
+  and without blocks, on odd grids, one-frame clips and other patch shapes.
+* bf16 (tcgen05 GEMMs and attention, fp32 residual): rel-L2 <= 1e-2 on every
+  pixel, at small and full width, and on the head's ragged column tile.
+* E4M3 block projections: against the oracle's E4M3 block, the block's
+  bounds (3e-2).
+* The full 6 x 34 x 60 clip (12,240 cells, 21 frames of 544 x 960): the head
+  and unpatchify checked on sampled cells that the oracle computes one by one,
+  one full-width block checked on sampled cells (the oracle's block restricted
+  to those rows), and the 26-layer decoder finite with every pixel written.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from oracle import decoder as D
+from oracle import fp8 as Q
+from few_step_dit_b200 import api, build, lib as L
+from few_step_dit_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    L.load()
+    yield
+    torch.cuda.synchronize()
+    api.device_error()
+
+
+def _run(w, n_layers=None, fp8=False, seed=None):
+    layers, io = S.make_decoder_weights(w, n_layers=n_layers, **({} if seed is None else {"seed": seed}))
+    lat = S.make_decoder_latents(w)
+    dl = [api.BlockWeights(api.quantize_block_weights({k: v.to(DEV) for k, v in l.items()})) if fp8 else
+          api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers]
+    dec = api.Decoder(api.dims_of(w, proj_fp8=fp8), dl,
+                      api.DecoderIO({k: v.to(DEV) for k, v in io.items()}, w.c_pix, w.patch_t, w.patch_s))
+    px = dec.forward(lat.to(DEV), w.grid)
+    torch.cuda.synchronize()
+    return px.double().cpu().numpy(), layers, io, lat
+
+
+def _oracle(w, layers, io, lat, block_fn=O.dit_block):
+    T, H, W = w.grid
+    return D.decoder_forward(lat.double().numpy(), [S.to_numpy64(l) for l in layers], S.to_numpy64(io), T, H, W,
+                             w.heads, w.head_dim, w.c_pix, w.patch_t, w.patch_s, block_fn=block_fn)
+
+
+TINY = S.DECODER_WORKLOADS["tiny_decoder_f32"]
+
+
+@pytest.mark.parametrize("kw", [{}, {"n_layers": 0}, {"grid": (1, 3, 7)}, {"grid": (2, 5, 3), "patch_t": 1},
+                                {"patch_s": 8, "c_pix": 1, "patch_t": 2}, {"grid": (4, 1, 1), "c_lat": 64}])
+def test_fp32_decoder_matches_oracle(kw):
+    w = S.scaled(TINY, **kw)
+    got, layers, io, lat = _run(w)
+    ref = _oracle(w, layers, io, lat)
+    assert got.shape == ref.shape == w.pixel_shape
+    assert O.rel_l2(got, ref) < 1e-5
+
+
+@pytest.mark.parametrize("kw", [{"grid": (3, 9, 10), "patch_s": 16},                  # 270 cells, 3,072 columns
+                                {"grid": (2, 7, 11), "patch_s": 4, "c_pix": 1, "patch_t": 1},  # 16 columns
+                                {"grid": (1, 12, 12), "patch_s": 8}])                # one frame
+def test_bf16_decoder_matches_oracle(kw):
+    w = S.scaled(TINY, dtype="bf16", **kw)
+    got, layers, io, lat = _run(w)
+    ref = _oracle(w, layers, io, lat)
+    assert O.rel_l2(got, ref) < 1e-2
+
+
+def test_bf16_full_width_decoder_two_layers():
+    # hidden 2048, 16 heads, FFN 8192 on a 3 x 17 x 30 grid (1,530 cells)
+    w = S.scaled(S.DECODER_WORKLOADS["decoder_6x34x60"], grid=(3, 17, 30))
+    got, layers, io, lat = _run(w, n_layers=2)
+    ref = _oracle(w, layers, io, lat)
+    assert O.rel_l2(got, ref) < 1e-2
+
+
+def test_fp8_decoder_matches_fp8_oracle():
+    w = S.scaled(TINY, dtype="bf16", grid=(3, 9, 10), patch_s=8)
+    got, layers, io, lat = _run(w, fp8=True)
+    ref = _oracle(w, layers, io, lat, block_fn=Q.dit_block_fp8)
+    assert O.rel_l2(got, ref) < 3e-2
+
+
+FULL = S.DECODER_WORKLOADS["decoder_6x34x60"]
+
+
+def _sample_cells(w, seed=5):
+    T, H, W = w.grid
+    corners = [0, W - 1, (H - 1) * W, H * W - 1, H * W, w.n_cells - 1, w.n_cells - W]
+    return np.unique(np.concatenate([corners, np.random.default_rng(seed).integers(0, w.n_cells, 24)]))
+
+
+def _cell_pixels(w, px, cell):
+    """The pixels cell `cell` wrote, as [c_pix, patch frames, ps, ps]."""
+    T, H, W = w.grid
+    t, h, wc = cell // (H * W), (cell // W) % H, cell % W
+    ps, pt = w.patch_s, w.patch_t
+    f0 = max(0, pt * t - pt + 1)
+    return px[f0:pt * t + 1, :, h * ps:(h + 1) * ps, wc * ps:(wc + 1) * ps].transpose(1, 0, 2, 3)
+
+
+def _oracle_cell_pixels(w, y_row, cell):
+    T, H, W = w.grid
+    t = cell // (H * W)
+    p = y_row.reshape(w.c_pix, w.patch_t, w.patch_s, w.patch_s)
+    return p[:, w.patch_t - 1:] if t == 0 else p
+
+
+@pytest.fixture(scope="module")
+def full_weights():
+    return S.make_decoder_weights(FULL, device=DEV, n_layers=1), S.make_decoder_latents(FULL, device=DEV)
+
+
+def _full_decoder(layers, io, n_layers):
+    bl = [api.BlockWeights(l) for l in layers[:n_layers]]
+    return api.Decoder(api.dims_of(FULL), bl, api.DecoderIO(io, FULL.c_pix, FULL.patch_t, FULL.patch_s))
+
+
+@pytest.mark.parametrize("n_layers", [0, 1])
+def test_full_clip_sampled_cells(full_weights, n_layers):
+    (layers, io), lat = full_weights
+    px = _full_decoder(layers, io, n_layers).forward(lat, FULL.grid)
+    torch.cuda.synchronize()
+    assert tuple(px.shape) == FULL.pixel_shape == (21, 3, 544, 960)
+    cells = _sample_cells(FULL)
+    px = px.double().cpu().numpy()
+    io64 = S.to_numpy64(io)
+    x = O.linear(lat.double().cpu().numpy(), io64["w_in"], io64["b_in"])
+    if n_layers:
+        x_rows = O.dit_block_rows(x, S.to_numpy64(layers[0]), D.grid_positions(*FULL.grid), FULL.heads,
+                                  FULL.head_dim, cells)
+    else:
+        x_rows = x[cells]
+    y = D.pixel_head(x_rows, io64)
+    got = np.concatenate([_cell_pixels(FULL, px, int(c)).ravel() for c in cells])
+    ref = np.concatenate([_oracle_cell_pixels(FULL, y[i], int(c)).ravel() for i, c in enumerate(cells)])
+    assert O.rel_l2(got, ref) < 1e-2
+
+
+def test_full_26_layer_decoder_writes_every_pixel():
+    layers, io = S.make_decoder_weights(FULL, device=DEV)
+    lat = S.make_decoder_latents(FULL, device=DEV)
+    dec = _full_decoder(layers, io, FULL.n_layers)
+    px = torch.full(FULL.pixel_shape, float("nan"), device=DEV)
+    dec.forward(lat, FULL.grid, pixels=px)
+    torch.cuda.synchronize()
+    assert torch.isfinite(px).all()
+    again = dec.forward(lat, FULL.grid)
+    torch.cuda.synchronize()
+    assert torch.equal(px, again)   # deterministic: no atomics on the path
