@@ -85,15 +85,17 @@ def rmsnorm_quant(x, g, eps=1e-6, stream=None):
     return q, s[:rows]
 
 
-def linear_fp8(dims, qa, sa, qw, sw, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, stream=None):
+def linear_fp8(dims, qa, sa, qw, sw, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, scratch=None,
+               stream=None):
     """E4M3 projection: epilogue((qa qw^T) * sa[row] * sw[col] + b)."""
     M, K = qa.shape
     N = qw.shape[0]
     if out is None:
         od = torch.float32 if epilogue in (L.EPI_RESIDUAL, L.EPI_BIAS_F32) else torch.bfloat16
         out = torch.empty(M, N, dtype=od, device=qa.device)
-    L.call("fsdit_linear_fp8", C.byref(dims), L.ptr(qa), L.ptr(sa), L.ptr(qw), L.ptr(sw), L.ptr(b), L.ptr(out),
-           L.ptr(resid), L.ptr(pos), M, N, K, epilogue, _stream(stream))
+    L.call("fsdit_linear_fp8_ws", C.byref(dims), L.ptr(qa), L.ptr(sa), L.ptr(qw), L.ptr(sw), L.ptr(b), L.ptr(out),
+           L.ptr(resid), L.ptr(pos), M, N, K, epilogue, L.ptr(scratch),
+           scratch.numel() if scratch is not None else 0, _stream(stream))
     return out
 
 
@@ -196,14 +198,22 @@ def rmsnorm_cast(x, g, eps=1e-6, stream=None):
     return xn
 
 
-def linear(dims, a, w, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, stream=None):
+def gemm_scratch(device):
+    """Caller scratch for the projections' tail cut (fsdit_gemm_scratch_size bytes)."""
+    return torch.empty(L.load().fsdit_gemm_scratch_size(), dtype=torch.uint8, device=device)
+
+
+def linear(dims, a, w, b, epilogue=L.EPI_BIAS, resid=None, pos=None, out=None, scratch=None, stream=None):
+    """out = epilogue(a w^T + b); with `scratch` (gemm_scratch) the last wave's
+    tiles may be cut along K (fsdit_linear_ws)."""
     M, K = a.shape
     N = w.shape[0]
     if out is None:
         od = torch.float32 if epilogue in (L.EPI_BIAS_F32, L.EPI_RESIDUAL) else a.dtype
         out = torch.empty(M, N, dtype=od, device=a.device)
-    L.call("fsdit_linear", C.byref(dims), L.ptr(a), L.ptr(w), L.ptr(b), L.ptr(out), L.ptr(resid),
-           L.ptr(pos), M, N, K, epilogue, _stream(stream))
+    L.call("fsdit_linear_ws", C.byref(dims), L.ptr(a), L.ptr(w), L.ptr(b), L.ptr(out), L.ptr(resid),
+           L.ptr(pos), M, N, K, epilogue, L.ptr(scratch), scratch.numel() if scratch is not None else 0,
+           _stream(stream))
     return out
 
 

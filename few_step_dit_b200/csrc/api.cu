@@ -49,6 +49,15 @@ ProfScope::ProfScope(int c, int k, double fl, double by, cudaStream_t s) : slot(
 ProfScope::~ProfScope() {
   if (slot >= 0) prof_record(g_prof.ev[2 * slot + 1], st);
 }
+void ProfScope::add_kernels(int k) {
+  if (slot >= 0) g_prof.kernels[slot] += k;
+}
+// The launch scope open on this thread (a projection's launcher adds the
+// second kernel of a tail cut to it).
+static thread_local ProfScope* t_scope = nullptr;
+void prof_add_kernels(int k) {
+  if (t_scope != nullptr) t_scope->add_kernels(k);
+}
 
 fsdit_status launch_keep_map(int T, int H, int W, int32_t* keep_idx, int32_t* near_idx, cudaStream_t st);
 fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_t* posc, const int32_t* keep_idx,
@@ -173,6 +182,8 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.row_scale = nullptr;
   e.col_scale = nullptr;
   e.up_h = e.up_w = e.up_c = e.up_pt = e.up_ps = 1;
+  e.split_part = nullptr;
+  e.split_cnt = nullptr;
   return e;
 }
 
@@ -187,8 +198,11 @@ fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, co
   const double by = ((double)M * K + (double)N * K) * s + (double)M * N * out_b +
                     (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
   ProfScope ps(prof_cls >= 0 ? prof_cls : cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);
-  if (d->dtype == FSDIT_BF16) return launch_linear_tc(a, w, ep, M, N, K, st);
-  return launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
+  t_scope = &ps;
+  const fsdit_status r = d->dtype == FSDIT_BF16 ? launch_linear_tc(a, w, ep, M, N, K, st)
+                                                : launch_linear_simt(FSDIT_F32, a, w, ep, M, N, K, st);
+  t_scope = nullptr;
+  return r;
 }
 
 fsdit_status launch_linear_fp8(const fsdit_dims* d, const uint8_t* qa, const void* qw, const EpiParams& ep, int M,
@@ -202,7 +216,10 @@ fsdit_status launch_linear_fp8(const fsdit_dims* d, const uint8_t* qa, const voi
                     (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
   ProfScope ps(cls, 1, 2.0 * M * N * K, by, st);
   (void)d;
-  return launch_linear_fp8_tc(qa, (const uint8_t*)qw, ep, M, N, K, st);
+  t_scope = &ps;
+  const fsdit_status r = launch_linear_fp8_tc(qa, (const uint8_t*)qw, ep, M, N, K, st);
+  t_scope = nullptr;
+  return r;
 }
 
 fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n, cudaStream_t st) {
@@ -576,9 +593,40 @@ fsdit_status fsdit_rmsnorm_cast(const float* x, const void* g, void* xn, int row
   return launch_rmsnorm_cast(x, g, xn, rows, hidden, eps, dtype, (cudaStream_t)stream);
 }
 
+size_t fsdit_gemm_scratch_size(void) { return SPLIT_WS_BYTES + SPLIT_CNT_BYTES; }
+
+}  // extern "C"
+
+namespace fsdit {
+// Point `ep` at caller scratch for the pair GEMM's tail cut and zero its
+// counters (nothing when scratch is null).
+static fsdit_status attach_scratch(EpiParams& ep, void* scratch, size_t bytes, cudaStream_t st) {
+  if (scratch == nullptr) return FSDIT_OK;
+  if (bytes < SPLIT_WS_BYTES + SPLIT_CNT_BYTES) {
+    set_error("GEMM scratch: need %zu bytes, got %zu", SPLIT_WS_BYTES + SPLIT_CNT_BYTES, bytes);
+    return FSDIT_E_WORKSPACE;
+  }
+  if (!aligned16(scratch)) {
+    set_error("GEMM scratch must be 16-byte aligned");
+    return FSDIT_E_ALIGN;
+  }
+  ep.split_part = (float*)scratch;
+  ep.split_cnt = (int*)((uint8_t*)scratch + SPLIT_WS_BYTES);
+  return cuda_check(cudaMemsetAsync(ep.split_cnt, 0, SPLIT_CNT_BYTES, st), "cudaMemsetAsync(GEMM scratch counters)");
+}
+}  // namespace fsdit
+
+extern "C" {
+
 fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, const void* b, void* out,
                           const float* resid, const int32_t* pos, int M, int N, int K, int epilogue,
                           fsdit_stream_t stream) {
+  return fsdit_linear_ws(dims, a, w, b, out, resid, pos, M, N, K, epilogue, nullptr, 0, stream);
+}
+
+fsdit_status fsdit_linear_ws(const fsdit_dims* dims, const void* a, const void* w, const void* b, void* out,
+                             const float* resid, const int32_t* pos, int M, int N, int K, int epilogue,
+                             void* scratch, size_t scratch_bytes, fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));
   FS_TRY(need(a, "a"));
   FS_TRY(need(w, "w"));
@@ -601,6 +649,7 @@ fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const void* w, 
     }
   }
   EpiParams ep = make_ep(dims, epilogue, b, out, N, resid, pos);
+  FS_TRY(attach_scratch(ep, scratch, scratch_bytes, (cudaStream_t)stream));
   return launch_linear(dims, a, w, ep, M, N, K, (cudaStream_t)stream);
 }
 
@@ -646,6 +695,13 @@ fsdit_status fsdit_rmsnorm_quant(const float* x, const void* g, int rows, int hi
 fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* qa, const float* sa, const uint8_t* qw,
                               const float* sw, const void* b, void* out, const float* resid, const int32_t* pos, int M,
                               int N, int K, int epilogue, fsdit_stream_t stream) {
+  return fsdit_linear_fp8_ws(dims, qa, sa, qw, sw, b, out, resid, pos, M, N, K, epilogue, nullptr, 0, stream);
+}
+
+fsdit_status fsdit_linear_fp8_ws(const fsdit_dims* dims, const uint8_t* qa, const float* sa, const uint8_t* qw,
+                                 const float* sw, const void* b, void* out, const float* resid, const int32_t* pos,
+                                 int M, int N, int K, int epilogue, void* scratch, size_t scratch_bytes,
+                                 fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));
   if (dims->dtype != FSDIT_BF16) {
     set_error("linear_fp8: dims.dtype must be FSDIT_BF16 (bias, outputs)");
@@ -681,6 +737,7 @@ fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* qa, const f
   EpiParams ep = make_ep(dims, epilogue, b, out, N, resid, pos);
   ep.row_scale = sa;
   ep.col_scale = sw;
+  FS_TRY(attach_scratch(ep, scratch, scratch_bytes, (cudaStream_t)stream));
   return launch_linear_fp8(dims, qa, qw, ep, M, N, K, (cudaStream_t)stream);
 }
 

@@ -70,7 +70,14 @@ struct EpiParams {
   const float* col_scale;  // row_scale[row] * col_scale[col] (FP8 dequantization) before the bias
   int up_h, up_w;          // EPI_UNPATCH: the rows are the cells of a (t, h, w) grid up_h x up_w per frame,
   int up_c, up_pt, up_ps;  // each column a pixel of the cell's up_c x up_pt x up_ps x up_ps patch
+  float* split_part;       // pair GEMM tail cut: caller scratch for the partial accumulators
+  int* split_cnt;          // (SPLIT_WS_BYTES) and its zeroed counters (SPLIT_CNT_BYTES), or null: no cut
 };
+
+// Scratch of the pair GEMM's tail cut: 128 units of 256 KB fp32 partials and
+// 64 x 16 int counters (zero between launches; each launch leaves them zero).
+constexpr size_t SPLIT_WS_BYTES = (size_t)128 << 18;
+constexpr size_t SPLIT_CNT_BYTES = 64 * 16 * 4;
 
 // Decoder pixel head (internal epilogue, not reachable through fsdit_linear):
 // out (f32) = acc + b written straight into frames [F][up_c][up_h*ps][up_w*ps].
@@ -329,9 +336,12 @@ enum ProfClass {
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);
   ~ProfScope();
+  void add_kernels(int k);
   int slot;
   cudaStream_t st;
 };
+// Count k more kernels in the projection launch scope open on this thread.
+void prof_add_kernels(int k);
 
 int num_sms();
 void set_error(const char* fmt, ...);

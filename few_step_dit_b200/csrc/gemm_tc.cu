@@ -36,6 +36,13 @@ struct Args {
   int M, N, K;
   int tiles_m, tiles_n, group_n;
   EpiParams ep;
+  // Split tail (pair kernel only): units [0, full_units) are whole tiles
+  // 0..full_units-1; every later tile is cut into `split` units along K
+  // (unit full_units + slot*split + s covers k-blocks [s*KB/split,
+  // (s+1)*KB/split) of tile full_units + slot).  split == 1: no tail cut.
+  int full_units, split, n_units;
+  float* part;  // [slot*split + s][16 regions][4 chunks][8][32 lanes] float4 partial accumulators
+  int* cnt;     // [slot][16 regions] arrivals, zero between launches
 };
 
 __device__ __forceinline__ void tile_coords(int tile, const Args& a, int& mb, int& nb) {
@@ -203,6 +210,32 @@ __global__ void __launch_bounds__(THREADS, 1)
 // per warp).
 namespace gemm2 {
 
+// Tail cut bounds: at most SPLIT_MAX_UNITS partial units (256 KB of fp32
+// partials each) and SPLIT_MAX_SLOTS cut tiles per launch.
+constexpr int SPLIT_MAX_UNITS = 128, SPLIT_MAX_SLOTS = 64, SPLIT_REGIONS = 16;
+constexpr int SPLIT_MIN_KB = 32, SPLIT_UNIT_KB = 12;
+
+// Tile, k-block range, part and tail slot of work unit u: a whole tile
+// (SPLIT = false: tile u) or part s of tail tile full_units + slot
+// (SPLIT = true: k-blocks [s*KB/split, (s+1)*KB/split)).
+template <bool SPLIT>
+__device__ __forceinline__ void unit_work(int u, const gemm::Args& a, int KB, int& tile, int& kb0, int& kb1,
+                                          int& s, int& slot) {
+  if constexpr (!SPLIT) {
+    tile = u;
+    kb0 = 0;
+    kb1 = KB;
+    s = 0;
+    slot = 0;
+  } else {
+    slot = u / a.split;
+    s = u - slot * a.split;
+    tile = a.full_units + slot;
+    kb0 = s * KB / a.split;
+    kb1 = (s + 1) * KB / a.split;
+  }
+}
+
 constexpr int BM = 256, BN = 256, BK = 64;  // BK: bf16 elements per stage row (128 bytes)
 constexpr int BK8 = 128;                     // E4M3 elements per stage row (128 bytes)
 constexpr int HM = BM / 2, HN = BN / 2;  // per-CTA share of A rows and B rows
@@ -222,9 +255,80 @@ constexpr int GROUP_N = 8;
 constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, 0);
 constexpr uint32_t IDESC_FP8 = ptx::idesc_e4m3(BM, BN);
 
+// Epilogue of one split unit, for one epilogue warp's region (its rank's rows
+// of one TMEM lane quarter, one column half): park this unit's fp32
+// accumulators of the region in the scratch, release the TMEM buffer (arrive
+// on `tempty`, rank 0's barrier: locally when `local`, else through the
+// cluster), count the part in; the warp that brings the region's last part
+// sums all parts in split order -- the same result whichever unit finishes
+// last -- runs the epilogue and clears the counter for the next launch.
+__device__ __forceinline__ void split_unit_epilogue(const gemm::Args& args, uint32_t t_row, int slot, int sp,
+                                                 int region, int row, bool row_ok, int nb, int c0, int lane,
+                                                 uint32_t tempty, bool local) {
+  using namespace ptx;
+  constexpr int CHUNKS = BN / 64;                 // 32-column chunks of a region
+  constexpr int REGION_F4 = CHUNKS * 8 * 32;      // float4s of one region's part
+  float4* mine = reinterpret_cast<float4*>(args.part) +
+                 ((size_t)(slot * args.split + sp) * SPLIT_REGIONS + region) * REGION_F4;
+#pragma unroll 1
+  for (int c = 0; c < CHUNKS; ++c) {
+    float v[32];
+    tmem_ld32(t_row + (uint32_t)((c0 + c) * 32), v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      mine[(c * 8 + i) * 32 + lane] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) {
+    if (local) mbar_arrive(tempty);
+    else mbar_arrive_cluster(tempty);
+  }
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  int* cnt = args.cnt + slot * SPLIT_REGIONS + region;
+  if (lane == 0) last = atomicAdd(cnt, 1) == args.split - 1 ? 1 : 0;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  const float4* parts = reinterpret_cast<const float4*>(args.part) +
+                        ((size_t)(slot * args.split) * SPLIT_REGIONS + region) * REGION_F4;
+#pragma unroll 1
+  for (int c = 0; c < CHUNKS; ++c) {
+    const int col = nb * BN + (c0 + c) * 32;
+    const bool full = row_ok && col + 32 <= args.N;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll 1
+    for (int p = 0; p < args.split; ++p) {
+      const float4* src = parts + (size_t)p * SPLIT_REGIONS * REGION_F4 + c * 8 * 32 + lane;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 t = __ldcg(src + i * 32);
+        v[4 * i] += t.x;
+        v[4 * i + 1] += t.y;
+        v[4 * i + 2] += t.z;
+        v[4 * i + 3] += t.w;
+      }
+    }
+    if (full) {
+      Epi32Pre pre;
+      epi32_prefetch(args.ep, row, col, pre);
+      epi32_apply(args.ep, row, col, v, pre);
+    } else if (row_ok && col < args.N) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 2)
+        if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
+    }
+  }
+  if (lane == 0) *cnt = 0;
+}
+
 // FP8 = true: E4M3 operands (kind::f8f6f4, 32 K elements per MMA), the same
 // 128-byte stage rows; the epilogue applies the per-row / per-column scales.
-template <bool FP8>
+template <bool FP8, bool SPLIT>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const gemm::Args args) {
@@ -273,7 +377,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int num_tiles = args.tiles_m * args.tiles_n;
   const int KB = (args.K + BKE - 1) / BKE;
 
   if (warp == 0) {
@@ -284,11 +387,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t last_ph = 0;
       bool ok = true;
       const uint32_t full0 = peer_addr(FULL(0), 0u);  // rank 0's full barriers
-      for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
-        int mb, nb;
+      for (int u = cid; u < args.n_units && ok; u += ncl) {
+        int tile, kb0, kb1, sp, slot, mb, nb;
+        unit_work<SPLIT>(u, args, KB, tile, kb0, kb1, sp, slot);
         gemm::tile_coords(tile, args, mb, nb);
         const int row_a = mb * BM + (int)rank * HM, row_b = nb * BN + (int)rank * HN;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(EMPTY(s), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + s * STAGE_BYTES;
           const uint32_t full = full0 + 8u * (uint32_t)s;
@@ -317,13 +421,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t ph = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++it) {
+      for (int u = cid; u < args.n_units && ok; u += ncl, ++it) {
+        int tile, kb0, kb1, sp, slot;
+        unit_work<SPLIT>(u, args, KB, tile, kb0, kb1, sp, slot);
         const int buf = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait_cluster(TEMPTY(buf), aph ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(FULL(s), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + s * STAGE_BYTES, sb = sa + A_BYTES;
@@ -332,12 +438,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int k = 0; k < 4 * BOXES; ++k) {
             const uint32_t oa = (uint32_t)((k >> 2) * (HM * 128) + (k & 3) * 32);
             const uint32_t ob = (uint32_t)((k >> 2) * (HN * 128) + (k & 3) * 32);
+            const uint32_t acc = (kb != kb0 || k != 0) ? 1u : 0u;
             if constexpr (FP8)
-              mma_e4m3_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC_FP8,
-                               (kb | k) != 0 ? 1u : 0u);
+              mma_e4m3_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC_FP8, acc);
             else
-              mma_bf16_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC,
-                               (kb | k) != 0 ? 1u : 0u);
+              mma_bf16_ss_pair(d, sw128_desc(sa + oa, 16, 1024), sw128_desc(sb + ob, 16, 1024), IDESC, acc);
           }
           tc_commit_pair(EMPTY(s));
           tc_commit_pair(empty_peer0 + 8u * (uint32_t)s);
@@ -356,8 +461,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;                    // TMEM lane quarter this warp may access
     const int c0 = ((warp - 2) >> 2) * (BN / 64);  // first of its BN/64 column chunks
     const uint32_t tempty0 = peer_addr(TEMPTY(0), 0u);
+    // this warp's region of a tile: its rank's rows of lane quarter q, its
+    // column half (the unit of the split-tail bookkeeping)
+    const int region = ((int)rank * 4 + q) * 2 + (c0 != 0 ? 1 : 0);
     int it = 0;
-    for (int tile = cid; tile < num_tiles; tile += ncl, ++it) {
+    for (int u = cid; u < args.n_units; u += ncl, ++it) {
+      int tile, kb0, kb1, sp, slot;
+      unit_work<SPLIT>(u, args, KB, tile, kb0, kb1, sp, slot);
       const int buf = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       int mb, nb;
@@ -370,6 +480,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int row = mb * BM + (int)rank * HM + q * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
       const bool row_ok = row < args.M;
+      if constexpr (SPLIT) {
+        split_unit_epilogue(args, t_row, slot, sp, region, row, row_ok, nb, c0, lane,
+                            rank == 0 ? TEMPTY(buf) : tempty0 + 8u * (uint32_t)buf, rank == 0);
+        continue;
+      }
 #pragma unroll 1
       for (int c = c0; c < c0 + BN / 64; ++c) {
         const int col = nb * BN + c * 32;
@@ -467,7 +582,8 @@ static int pair_clusters_resident() {
   static std::once_flag once;
   static int n = 0;
   std::call_once(once, [] {
-    for (auto fn : {gemm2::tc_gemm_pair_kernel<false>, gemm2::tc_gemm_pair_kernel<true>}) {
+    for (auto fn : {gemm2::tc_gemm_pair_kernel<false, false>, gemm2::tc_gemm_pair_kernel<true, false>,
+                    gemm2::tc_gemm_pair_kernel<false, true>, gemm2::tc_gemm_pair_kernel<true, true>}) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
         (void)cudaGetLastError();
@@ -486,7 +602,7 @@ static int pair_clusters_resident() {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel<false>, &cfg) == cudaSuccess) n = c;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel<false, false>, &cfg) == cudaSuccess) n = c;
     (void)cudaGetLastError();
   });
   return n;
@@ -511,22 +627,59 @@ static fsdit_status launch_linear_pair(const void* a, const void* w, const EpiPa
   args.group_n = GROUP_N < args.tiles_n ? GROUP_N : args.tiles_n;
   args.ep = ep;
   const int tiles = args.tiles_m * args.tiles_n;
-  const int ncl = tiles < clusters ? tiles : clusters;
+  // Tail cut: the R tiles of a partial last wave leave most CTA pairs idle;
+  // cut each into S units along K (S <= pairs / R) that run as a second
+  // launch of the SPLIT kernel, so the last wave is about 1/S of a tile
+  // long.  The whole tiles run in the first launch, whose kernel has no split
+  // code.  Only long K pays for the second launch and the fixup: at least
+  // SPLIT_MIN_KB k-blocks per tile and SPLIT_UNIT_KB per unit.
+  const int KB = (K + (fp8 ? BK8 : BK) * BOXES - 1) / ((fp8 ? BK8 : BK) * BOXES);
+  int R = 0, S = 1;
+  if (ep.split_part != nullptr && ep.split_cnt != nullptr && KB >= SPLIT_MIN_KB) {
+    R = tiles % clusters;
+    S = R > 0 ? clusters / R : 1;
+    if (S > KB / SPLIT_UNIT_KB) S = KB / SPLIT_UNIT_KB;
+    if (S > 8) S = 8;
+    if (R > 0 && R * S > SPLIT_MAX_UNITS) S = SPLIT_MAX_UNITS / R;
+    if (R == 0 || R > SPLIT_MAX_SLOTS || S < 2) {
+      R = 0;
+      S = 1;
+    }
+  }
+  args.full_units = tiles - R;
+  args.split = S;
+  args.part = ep.split_part;
+  args.cnt = ep.split_cnt;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * ncl);
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  if (fp8)
-    return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<true>, tmA, tmB, args), "tc_gemm_pair_kernel<fp8>");
-  return cuda_check(cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<false>, tmA, tmB, args), "tc_gemm_pair_kernel");
+  auto launch = [&](bool split, int units) -> fsdit_status {
+    args.n_units = units;
+    const int ncl = units < clusters ? units : clusters;
+    cfg.gridDim = dim3(2 * ncl);
+    cudaError_t e;
+    if (fp8)
+      e = split ? cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<true, true>, tmA, tmB, args)
+                : cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<true, false>, tmA, tmB, args);
+    else
+      e = split ? cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<false, true>, tmA, tmB, args)
+                : cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<false, false>, tmA, tmB, args);
+    return cuda_check(e, split ? "tc_gemm_pair_kernel (tail cut)" : "tc_gemm_pair_kernel");
+  };
+  if (args.full_units > 0) FS_TRY(launch(false, args.full_units));
+  if (R > 0) {
+    FS_TRY(launch(true, R * S));
+    if (args.full_units > 0) prof_add_kernels(1);
+  }
+  return FSDIT_OK;
 }
 
 // E4M3 projection: always on pair tiles (their epilogue applies the scales).

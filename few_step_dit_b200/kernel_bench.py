@@ -66,17 +66,18 @@ def case_gemm(a):
         if epi == L.EPI_QKV_ROPE else None
     od = torch.float32 if epi in (L.EPI_RESIDUAL, L.EPI_BIAS_F32) else torch.bfloat16
     out = torch.empty(a.M, a.N, dtype=od, device="cuda")
+    scr = api.gemm_scratch("cuda") if a.cut else None
     if a.fp8:
         dims8 = api.make_dims(5376, heads, 14336, L.BF16, proj_fp8=True)
         qx, sx = api.quantize_rows(x)
         qw, sw = api.quantize_rows(w)
-        fn = lambda: api.linear_fp8(dims8, qx, sx, qw, sw, b, epi, resid=resid, pos=pos, out=out)
+        fn = lambda: api.linear_fp8(dims8, qx, sx, qw, sw, b, epi, resid=resid, pos=pos, out=out, scratch=scr)
     else:
-        fn = lambda: api.linear(dims, x, w, b, epi, resid=resid, pos=pos, out=out)
+        fn = lambda: api.linear(dims, x, w, b, epi, resid=resid, pos=pos, out=out, scratch=scr)
     ms = time_it(fn, a.iters, a.warmup)
     fl = 2.0 * a.M * a.N * a.K
-    return {"case": "gemm", "M": a.M, "N": a.N, "K": a.K, "epi": a.epi, "fp8": bool(a.fp8), "ms": ms,
-            "tflops": fl / ms / 1e9}
+    return {"case": "gemm", "M": a.M, "N": a.N, "K": a.K, "epi": a.epi, "fp8": bool(a.fp8), "tail_cut": bool(a.cut),
+            "ms": ms, "tflops": fl / ms / 1e9}
 
 
 def case_block(a):
@@ -276,6 +277,7 @@ def main():
     p.add_argument("--fp8", action="store_true",
                    help="gemm / chunk / decoder / generate: E4M3 projections (per-row scales)")
     p.add_argument("--grid", default="", help="chunk / decoder: latent grid TxHxW (default 6x34x60)")
+    p.add_argument("--cut", action="store_true", help="gemm: cut the last wave's tiles along K (fsdit_linear_ws)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()

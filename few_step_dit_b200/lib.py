@@ -124,6 +124,10 @@ _SIGS = {
     "fsdit_history_gather": (_I, [C.POINTER(HistoryStore), C.POINTER(HistoryEntry), _I, _P, _I, _P, _P]),
     "fsdit_history_copy_frame": (_I, [C.POINTER(HistoryStore), _I, _P, _P]),
     "fsdit_chunk_tags": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "fsdit_gemm_scratch_size": (C.c_size_t, []),
+    "fsdit_linear_ws": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, C.c_size_t, _P]),
+    "fsdit_linear_fp8_ws": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, C.c_size_t,
+                                 _P]),
     "fsdit_decoder_frames": (_I, [_I, _I]),
     "fsdit_decoder_workspace_size": (C.c_size_t, [C.POINTER(Dims), C.POINTER(DecoderIO), _I, _I, _I]),
     "fsdit_decoder_forward": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(DecoderIO), _I, _I,

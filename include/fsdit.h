@@ -270,6 +270,33 @@ FSDIT_API fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* q
                                         const int32_t* pos, int M, int N, int K, int epilogue,
                                         fsdit_stream_t stream);
 
+/* Tail cut of the tensor-core projections.  A projection runs as a
+ * persistent grid of CTA pairs over 256 x 256 output tiles; when the tiles
+ * leave the last wave mostly idle (R tiles left for P pairs, R <= P/2), the
+ * *_ws calls cut each of those R tiles along K into S <= P/R units (at least
+ * four 128-byte K steps each, at most 8) that run on the idle pairs.  Each
+ * unit parks its fp32 partial accumulators in `scratch`; the unit that
+ * completes a tile region last sums the parts in unit order (so the result
+ * does not depend on which unit finishes last) and applies the epilogue.
+ * scratch (device, 16-byte aligned) holds fsdit_gemm_scratch_size() bytes;
+ * the call first zeroes its counters (one memset on `stream`); NULL scratch
+ * = the plain call.  Only GEMMs of at least 32 K steps are cut, into units
+ * of at least 12.  Same arguments and errors as fsdit_linear /
+ * fsdit_linear_fp8, plus FSDIT_E_WORKSPACE / FSDIT_E_ALIGN for the scratch.
+ * The cut shortens a GEMM run on its own (measured 16-30% on the compressed
+ * Flash projections); inside a long power-capped pass the GPU's clock, not
+ * its idle SMs, sets the time and the cut gains nothing, so the block,
+ * stack, sampler and decoder calls run whole tiles only. */
+FSDIT_API size_t fsdit_gemm_scratch_size(void);
+FSDIT_API fsdit_status fsdit_linear_ws(const fsdit_dims* dims, const void* a, const void* w, const void* b,
+                                       void* out, const float* resid, const int32_t* pos, int M, int N, int K,
+                                       int epilogue, void* scratch, size_t scratch_bytes, fsdit_stream_t stream);
+FSDIT_API fsdit_status fsdit_linear_fp8_ws(const fsdit_dims* dims, const uint8_t* qa, const float* sa,
+                                           const uint8_t* qw, const float* sw, const void* b, void* out,
+                                           const float* resid, const int32_t* pos, int M, int N, int K,
+                                           int epilogue, void* scratch, size_t scratch_bytes,
+                                           fsdit_stream_t stream);
+
 /* Joint attention ([tokendh] backbone section: one sequence of text,
  * video and audio tokens through one denoiser): for each head,
  * softmax(q k^T / sqrt(128)) v over all n rows, no mask.  With A = heads*128:
