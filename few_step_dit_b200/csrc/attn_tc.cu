@@ -94,36 +94,6 @@ __device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b) {
-  f2_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// 2^x for a pair on the FMA pipe, x <= 0: x = j + f with j = round(x) (the
-// 1.5 * 2^23 shifter leaves j in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f from a cubic fitted to 2^f on that interval (relative error below
-// 7.5e-5, far under the bf16 rounding P gets next); j is added to the exponent
-// field as an integer.  Inputs below -125 are clamped (their 2^x underflows
-// bf16 P anyway).
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  const f2_t x = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const f2_t shifter = f2(12582912.0f, 12582912.0f);
-  const f2_t t = f2_add(x, shifter);
-  const f2_t fr = f2_sub(x, f2_sub(t, shifter));
-  f2_t q = f2_fma(f2(0.0551716577f, 0.0551716577f), fr, f2(0.242611121f, 0.242611121f));
-  q = f2_fma(q, fr, f2(0.693260988f, 0.693260988f));
-  q = f2_fma(q, fr, f2(0.999928074f, 0.999928074f));
-  float t0, t1, q0, q1;
-  f2_split(t, t0, t1);
-  f2_split(q, q0, q1);
-  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
-// One pair in EMU_EVERY is exponentiated on the FMA pipe (0: none), taking
-// that share of the work off the MUFU pipe.
-constexpr int EMU_EVERY = 0;
 
 // O (+)= P V with P [128 x 16k] in TMEM (A operand) and V in shared memory.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -315,14 +285,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pk[BKV / 2];
 #pragma unroll
       for (int c = 0; c < BKV; c += 2) {
-        float x0, x1, p0, p1;
+        float x0, x1;
         f2_split(f2_fma(f2(s[c], s[c + 1]), scale2, negm2), x0, x1);
-        if (EMU_EVERY > 0 && (c >> 1) % (EMU_EVERY > 0 ? EMU_EVERY : 1) == EMU_EVERY - 1) {
-          exp2_poly_pair(x0, x1, p0, p1);
-        } else {
-          p0 = ex2(x0);
-          p1 = ex2(x1);
-        }
+        const float p0 = ex2(x0), p1 = ex2(x1);
         acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2(p0, p1));
         pk[c >> 1] = pack_bf16(p0, p1);
       }

@@ -12,7 +12,7 @@ Sources:
 * [ananclaw explainer] section 3.4 "推理加速": the Flash model runs with a
   lightweight VAE decoder.
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
 
 * Architecture.  The pages give depth, width and FFN ratio only; "hidden
   width" and "feed-forward expansion" are transformer terms, so the decoder

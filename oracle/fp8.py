@@ -5,7 +5,7 @@ Source: [PaperDaily] section 二 "Flash怎么把22帧压到377毫秒", third ste
 model switches suitable projection layers to low-bit weights and activations
 and fuses normalization, quantization, RoPE and the residual update into the
 surrounding computation.  The pages give no format or scaling, so every choice
-below is a reading (each also listed in the design doc):
+below is a reading:
 
 * Format: FP8 E4M3 (OCP "E4M3FN": 1 sign, 4 exponent bits with bias 7, 3
   mantissa bits, subnormals, no infinity, largest finite 448).  Rounding is to

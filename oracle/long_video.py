@@ -16,7 +16,7 @@ Sources:
   storage is bounded too: once full, the initial frame and the most recent
   frames are kept and the middle entries dropped.
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
 
 * Stride-s sampling of a latent frame keeps the positions whose row and
   column are both multiples of s (no extra edge row/column: the pages state
