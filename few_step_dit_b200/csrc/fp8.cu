@@ -3,9 +3,10 @@
 // next to the normalization).
 //
 // One fp32 scale per row: s = amax / 448 (1 for an all-zero row) and codes
-// E4M3(v / s), round to nearest even, saturating; amax, the IEEE division and
-// the rounding happen in fp32.  Activations are quantized per token, weights
-// per output channel (rows of [N, K]).
+// E4M3(v * r) with r = 1 / s rounded to fp32 once per row (IEEE reciprocal),
+// round to nearest even, saturating; amax, the reciprocal, the product and the
+// rounding happen in fp32.  Activations are quantized per token, weights per
+// output channel (rows of [N, K]).
 
 namespace fsdit {
 namespace q8 {
@@ -50,10 +51,77 @@ template <> __device__ __forceinline__ void load8<bf16>(const bf16* p, float* v)
   }
 }
 
-// One 256-thread block per row: amax pass, then the codes (cols % 8 == 0).
-template <typename T>
+// 8 codes of v[0..7] * rs (rs: the fp32 reciprocal of the row scale) as one
+// 8-byte word.
+__device__ __forceinline__ uint2 codes8(const float* v, float rs) {
+  uint2 out;
+  out.x = (uint32_t)e4m3x2(__fmul_rn(v[0], rs), __fmul_rn(v[1], rs)) |
+          ((uint32_t)e4m3x2(__fmul_rn(v[2], rs), __fmul_rn(v[3], rs)) << 16);
+  out.y = (uint32_t)e4m3x2(__fmul_rn(v[4], rs), __fmul_rn(v[5], rs)) |
+          ((uint32_t)e4m3x2(__fmul_rn(v[6], rs), __fmul_rn(v[7], rs)) << 16);
+  return out;
+}
+
+// 8 raw input values of a row kept in registers between the amax pass and
+// the codes: packed for bf16 (16 bytes), as fp32 otherwise.
+template <typename T> struct Raw8;
+template <> struct Raw8<bf16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const bf16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ void get(float* v) const { load8<bf16>(reinterpret_cast<const bf16*>(&u), v); }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = *reinterpret_cast<const float4*>(p);
+    b = *reinterpret_cast<const float4*>(p + 4);
+  }
+  __device__ __forceinline__ void get(float* v) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// One 256-thread block per row (cols % 8 == 0, cols <= 256 * 8 * CH): the
+// row is read once into registers, reduced to its amax, then turned into
+// codes.
+template <typename T, int CH>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int cols, uint8_t* __restrict__ q,
                                                          float* __restrict__ s) {
+  __shared__ float red[8];
+  const int r = blockIdx.x;
+  const T* ar = a + (size_t)r * cols;
+  Raw8<T> raw[CH];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = (threadIdx.x + k * 256) * 8;
+    if (c < cols) {
+      raw[k].load(ar + c);
+      float v[8];
+      raw[k].get(v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+  }
+  const float sc = row_scale(block_max(amax, red));
+  if (threadIdx.x == 0) s[r] = sc;
+  const float rs = __frcp_rn(sc);
+  uint8_t* qr = q + (size_t)r * cols;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = (threadIdx.x + k * 256) * 8;
+    if (c < cols) {
+      float v[8];
+      raw[k].get(v);
+      *reinterpret_cast<uint2*>(qr + c) = codes8(v, rs);
+    }
+  }
+}
+
+// Rows longer than 256 * 8 * 8 values: two passes over the row.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_long_kernel(const T* __restrict__ a, int cols,
+                                                              uint8_t* __restrict__ q, float* __restrict__ s) {
   __shared__ float red[8];
   const int r = blockIdx.x;
   const T* ar = a + (size_t)r * cols;
@@ -66,16 +134,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
   }
   const float sc = row_scale(block_max(amax, red));
   if (threadIdx.x == 0) s[r] = sc;
+  const float rs = __frcp_rn(sc);
   uint8_t* qr = q + (size_t)r * cols;
   for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
     float v[8];
     load8<T>(ar + c, v);
-    uint2 out;
-    out.x = (uint32_t)e4m3x2(__fdiv_rn(v[0], sc), __fdiv_rn(v[1], sc)) |
-            ((uint32_t)e4m3x2(__fdiv_rn(v[2], sc), __fdiv_rn(v[3], sc)) << 16);
-    out.y = (uint32_t)e4m3x2(__fdiv_rn(v[4], sc), __fdiv_rn(v[5], sc)) |
-            ((uint32_t)e4m3x2(__fdiv_rn(v[6], sc), __fdiv_rn(v[7], sc)) << 16);
-    *reinterpret_cast<uint2*>(qr + c) = out;
+    *reinterpret_cast<uint2*>(qr + c) = codes8(v, rs);
   }
 }
 
@@ -113,13 +177,14 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const float* __restr
   }
   const float sc = row_scale(block_max(amax, red2));
   if (threadIdx.x == 0) s[r] = sc;
+  const float rs = __frcp_rn(sc);
   uint32_t* qr = reinterpret_cast<uint32_t*>(q + (size_t)r * hidden);
 #pragma unroll
   for (int k = 0; k < RMS_MAXV; ++k) {
     const int i = threadIdx.x + k * 256;
     if (i < h4)
-      qr[i] = (uint32_t)e4m3x2(__fdiv_rn(v[k].x, sc), __fdiv_rn(v[k].y, sc)) |
-              ((uint32_t)e4m3x2(__fdiv_rn(v[k].z, sc), __fdiv_rn(v[k].w, sc)) << 16);
+      qr[i] = (uint32_t)e4m3x2(__fmul_rn(v[k].x, rs), __fmul_rn(v[k].y, rs)) |
+              ((uint32_t)e4m3x2(__fmul_rn(v[k].z, rs), __fmul_rn(v[k].w, rs)) << 16);
   }
 }
 
@@ -127,19 +192,28 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const float* __restr
 
 fsdit_status launch_quant_rows(const void* a, int dtype, int rows, int cols, uint8_t* q, float* s, cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
-  ProfScope ps(PC_QUANT, 1, 0.0, (double)rows * cols * (dtype == FSDIT_BF16 ? 2.0 : 4.0) * 2.0 + (double)rows * cols,
+  ProfScope ps(PC_QUANT, 1, 0.0, (double)rows * cols * (dtype == FSDIT_BF16 ? 2.0 : 4.0) + (double)rows * (cols + 4),
                st);
-  if (dtype == FSDIT_BF16)
-    q8::quant_rows_kernel<bf16><<<rows, 256, 0, st>>>((const bf16*)a, cols, q, s);
-  else
-    q8::quant_rows_kernel<float><<<rows, 256, 0, st>>>((const float*)a, cols, q, s);
+  // register-resident rows of up to 2048 * CH values, CH a power of two
+  const int ch = (cols + 2047) / 2048;
+  auto go = [&](auto tag) {
+    using T = decltype(tag);
+    const T* p = (const T*)a;
+    if (ch <= 1) q8::quant_rows_kernel<T, 1><<<rows, 256, 0, st>>>(p, cols, q, s);
+    else if (ch <= 2) q8::quant_rows_kernel<T, 2><<<rows, 256, 0, st>>>(p, cols, q, s);
+    else if (ch <= 4) q8::quant_rows_kernel<T, 4><<<rows, 256, 0, st>>>(p, cols, q, s);
+    else if (ch <= 8) q8::quant_rows_kernel<T, 8><<<rows, 256, 0, st>>>(p, cols, q, s);
+    else q8::quant_rows_long_kernel<T><<<rows, 256, 0, st>>>(p, cols, q, s);
+  };
+  if (dtype == FSDIT_BF16) go(bf16());
+  else go(float());
   return cuda_check(cudaGetLastError(), "quant_rows_kernel");
 }
 
 fsdit_status launch_rmsnorm_quant(const float* x, const void* g, int rows, int hidden, float eps, uint8_t* q, float* s,
                                   cudaStream_t st) {
   if (rows <= 0) return FSDIT_OK;
-  ProfScope ps(PC_NORM, 1, 0.0, (double)rows * hidden * 5.0, st);
+  ProfScope ps(PC_NORM, 1, 0.0, (double)rows * (hidden * 5.0 + 4.0), st);
   q8::rmsnorm_quant_kernel<<<rows, 256, 0, st>>>(x, (const bf16*)g, hidden, eps, q, s);
   return cuda_check(cudaGetLastError(), "rmsnorm_quant_kernel");
 }

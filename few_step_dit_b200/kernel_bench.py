@@ -117,6 +117,13 @@ def case_memory(a):
     res["broadcast_gbs"] = (w.n_video + xc.shape[0] + n) * hb / ms / 1e6
     ms = time_it(lambda: api.rmsnorm_cast(x, gain), a.iters, a.warmup)
     res["rmsnorm_ms"], res["rmsnorm_gbs"] = ms, n * w.hidden * 6.0 / ms / 1e6
+    # E4M3 quantizers: the fused RMSNorm-quantizer (fp32 in, codes + scales out)
+    # and the per-row quantizer of a bf16 attention output [n, A]
+    ms = time_it(lambda: api.rmsnorm_quant(x, gain), a.iters, a.warmup)
+    res["rmsnorm_quant_ms"], res["rmsnorm_quant_gbs"] = ms, n * (w.hidden * 5.0 + 4) / ms / 1e6
+    att = torch.randn(n, w.attn_dim, generator=g, device="cuda").bfloat16()
+    ms = time_it(lambda: api.quantize_rows(att), a.iters, a.warmup)
+    res["quant_rows_ms"], res["quant_rows_gbs"] = ms, n * (w.attn_dim * 3.0 + 4) / ms / 1e6
     return res
 
 

@@ -12,9 +12,13 @@ below is a reading:
   nearest with ties to even; magnitudes beyond 448 saturate to 448.
 * Scaling: one fp32 scale per row of the operand that is quantized -- per
   token for activations, per output channel for weights: s = amax / 448 (1
-  for an all-zero row), q = E4M3(value / s).  The amax, the division and the
-  rounding decision are taken in fp32 (the kernels' precision), so both sides
-  produce the same codes from the same fp32 inputs.
+  for an all-zero row), q = E4M3(value * r) with r = 1 / s, the scale's
+  reciprocal rounded to fp32 once per row (one multiply per value instead of
+  a division).  The amax, the reciprocal, the product and the rounding
+  decision are taken in fp32 (the kernels' precision), so both sides produce
+  the same codes from the same fp32 inputs; next to the exact quotient a
+  code moves only where value * r and value / s straddle an E4M3 rounding
+  midpoint (about 2^-20 of the values), by one step.
 * Which projections: the four of every block (QKV, O, FFN up, FFN down); the
   input/output embeddings, the time MLP and the heads stay as they are.
 * GEMM: out = (sum_k q_a q_w) * s_a[row] * s_w[col] + bias, then the
@@ -64,7 +68,8 @@ def quantize_rows(a):
     a32 = np.asarray(a, dtype=F32)
     amax = np.max(np.abs(a32), axis=1) if a32.shape[1] else np.zeros(a32.shape[0], F32)
     s = np.where(amax > 0, amax / F32(E4M3_MAX), F32(1.0)).astype(F32)
-    q = e4m3((a32 / s[:, None]).astype(F32))
+    r = (F32(1.0) / s).astype(F32)
+    q = e4m3((a32 * r[:, None]).astype(F32))
     return q, s.astype(F64)
 
 

@@ -46,7 +46,7 @@ def _values_to_codes(v):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("rows,cols", [(7, 256), (300, 5376), (33, 14336), (1, 16)])
+@pytest.mark.parametrize("rows,cols", [(7, 256), (300, 5376), (33, 14336), (1, 16), (4, 4096), (3, 16400)])
 def test_quantize_rows_bit_exact(dtype, rows, cols):
     g = torch.Generator().manual_seed(1)
     a = torch.randn(rows, cols, generator=g) * torch.exp(torch.randn(rows, 1, generator=g) * 2)

@@ -68,6 +68,20 @@ def test_quantize_rows_invariants():
     np.testing.assert_array_equal(s.astype(np.float32).astype(np.float64), s)
 
 
+def test_quantize_rows_reciprocal_codes_are_the_exact_quotients_codes_but_at_midpoints():
+    # the codes come from value * fp32(1/s); against the E4M3 rounding of the
+    # exact quotient value / s (computed in float64) a code may differ only
+    # where the two straddle a rounding midpoint: rarely, and by one step
+    rng = np.random.default_rng(11)
+    a = (rng.standard_normal((200, 4096)) * rng.uniform(0.01, 50, (200, 1))).astype(np.float32)
+    q, s = Q.quantize_rows(a)
+    exact = Q.e4m3(a.astype(np.float64) / s[:, None])
+    diff = q != exact
+    assert diff.mean() < 1e-4
+    step = np.maximum(np.abs(exact[diff]) * 2.0 ** -3, 2.0 ** -9)
+    assert (np.abs(q[diff] - exact[diff]) <= step * (1 + 1e-9)).all()
+
+
 def test_linear_fp8_exact_on_representable_operands():
     rng = np.random.default_rng(4)
     # entries from E4M3 integers; each row holds 448 so its scale is exactly 1
