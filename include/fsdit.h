@@ -279,8 +279,9 @@ FSDIT_API fsdit_status fsdit_linear_fp8(const fsdit_dims* dims, const uint8_t* q
  * completes a tile region last sums the parts in unit order (so the result
  * does not depend on which unit finishes last) and applies the epilogue.
  * scratch (device, 16-byte aligned) holds fsdit_gemm_scratch_size() bytes;
- * the call first zeroes its counters (one memset on `stream`); NULL scratch
- * = the plain call.  Only GEMMs of at least 32 K steps are cut, into units
+ * the call first zeroes its counters (one memset on `stream`), so calls that
+ * may run at the same time (other streams) need scratch of their own; NULL
+ * scratch = the plain call.  Only GEMMs of at least 32 K steps are cut, into units
  * of at least 12.  Same arguments and errors as fsdit_linear /
  * fsdit_linear_fp8, plus FSDIT_E_WORKSPACE / FSDIT_E_ALIGN for the scratch.
  * The cut shortens a GEMM run on its own (measured 16-30% on the compressed
