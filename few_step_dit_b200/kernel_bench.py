@@ -242,10 +242,12 @@ def case_decoder(a):
 
 
 def case_generate(a):
-    """The pages' latency protocol on one GPU: the 3-evaluation Flash
-    backbone pass (42 layers, 6x34x60, text 256, audio 64) followed by the
-    26-layer decoder of its video latents, one CUDA graph, warm."""
-    wb = S.WORKLOADS["flash_backbone_6x34x60"]
+    """The pages' latency protocol on one GPU: a sampling pass of the backbone
+    (default the 3-evaluation Flash pass, 42 layers, 6x34x60, text 256, audio
+    64; --backbone standard_backbone_12x34x60 for the 4-evaluation standard
+    model) followed by the 26-layer decoder of its target-grid video latents,
+    one CUDA graph, warm."""
+    wb = S.WORKLOADS[a.backbone]
     layers, io = S.make_weights(wb, device="cuda")
     if a.fp8:
         layers = [api.quantize_block_weights(l) for l in layers]
@@ -253,20 +255,23 @@ def case_generate(a):
                       wb.compress)
     seq = api.Sequence.from_workload(wb, S.pack_tokens(wb), "cuda")
     inp = S.make_inputs(wb, device="cuda")
+    a.grid = "x".join(str(v) for v in wb.grid)
     wd, dec = _decoder(a)
     assert wd.grid == wb.grid and wd.c_lat == wb.video_ch
     vl, al = inp["video_lat"].clone(), inp["audio_lat"].clone()
+    target = vl[:wb.n_video]  # the target grid's latents (control frames follow)
     px = torch.empty(wd.pixel_shape, device="cuda")
 
     def step():
         vl.copy_(inp["video_lat"])
         al.copy_(inp["audio_lat"])
         bb.sample(seq, wb.video_clock, wb.audio_clock, vl, inp["text_emb"], al)
-        dec.forward(vl, wd.grid, pixels=px)
+        dec.forward(target, wd.grid, pixels=px)
 
     ms = _graph_ms(step, a)
-    ms_dec = _graph_ms(lambda: dec.forward(vl, wd.grid, pixels=px), a)
-    return {"case": "generate", "workload": "flash_backbone_6x34x60+decoder_6x34x60", "fp8": bool(a.fp8),
+    ms_dec = _graph_ms(lambda: dec.forward(target, wd.grid, pixels=px), a)
+    T, H, W = wd.grid
+    return {"case": "generate", "workload": f"{wb.name}+decoder_{T}x{H}x{W}", "fp8": bool(a.fp8),
             "ms": ms, "ms_decoder": ms_dec, "ms_backbone": ms - ms_dec, "frames": wd.n_frames,
             "frames_per_s": wd.n_frames / ms * 1e3}
 
@@ -285,6 +290,7 @@ def main():
                    help="gemm / chunk / decoder / generate: E4M3 projections (per-row scales)")
     p.add_argument("--grid", default="", help="chunk / decoder: latent grid TxHxW (default 6x34x60)")
     p.add_argument("--cut", action="store_true", help="gemm: cut the last wave's tiles along K (fsdit_linear_ws)")
+    p.add_argument("--backbone", default="flash_backbone_6x34x60", help="generate: the backbone workload")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
