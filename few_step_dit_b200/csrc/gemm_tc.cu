@@ -36,10 +36,11 @@ struct Args {
   int M, N, K;
   int tiles_m, tiles_n, group_n;
   EpiParams ep;
-  // Split tail (pair kernel only): units [0, full_units) are whole tiles
-  // 0..full_units-1; every later tile is cut into `split` units along K
-  // (unit full_units + slot*split + s covers k-blocks [s*KB/split,
-  // (s+1)*KB/split) of tile full_units + slot).  split == 1: no tail cut.
+  // Tail cut (pair kernel only): tiles [0, full_units) run whole in the
+  // first launch (n_units = full_units); every later tile is cut into
+  // `split` units along K run by the SPLIT launch (n_units = cut tiles *
+  // split; unit slot*split + s covers k-blocks [s*KB/split, (s+1)*KB/split)
+  // of tile full_units + slot).  split == 1: no tail cut.
   int full_units, split, n_units;
   float* part;  // [slot*split + s][16 regions][4 chunks][8][32 lanes] float4 partial accumulators
   int* cnt;     // [slot][16 regions] arrivals, zero between launches
