@@ -137,3 +137,18 @@ def test_decoder_forward_rejects_bad_arguments_without_launching(fs):
     assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, odd, fake, big, None) == -3
     assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, fake, fake, 1024, None) == -6
     assert "workspace" in L.last_error()
+
+
+def test_linear_ws_rejects_bad_scratch_without_launching(fs):
+    d = _dims()
+    fake, odd = C.c_void_p(0x10000), C.c_void_p(0x10004)
+    need = fs.fsdit_gemm_scratch_size()
+    assert need >= 128 * 256 * 1024                          # 128 parts of 256 KB + counters
+    f = fs.fsdit_linear_ws
+    assert f(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 64, 0, fake, need - 1, None) == -6
+    assert "scratch" in L.last_error()
+    assert f(C.byref(d), fake, fake, fake, fake, None, None, 8, 64, 64, 0, odd, need, None) == -3
+    assert f(C.byref(d), fake, fake, fake, fake, None, None, 8, 60, 64, 0, fake, need, None) == -2
+    d8 = api.make_dims(5376, 42, 14336, L.BF16, proj_fp8=True)
+    g = fs.fsdit_linear_fp8_ws
+    assert g(C.byref(d8), fake, fake, fake, fake, fake, fake, None, None, 8, 64, 64, 0, fake, need - 1, None) == -6
