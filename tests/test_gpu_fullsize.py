@@ -137,3 +137,31 @@ def test_standard_four_eval_sampler_moves_only_target_rows():
     # control rows are clean conditions: untouched by all 4 Euler steps
     ctrl = slice(w.n_video, w.n_video + w.n_control)
     assert np.array_equal(got[ctrl], inp["video_lat"].double().numpy()[ctrl])
+
+
+def test_flash_pass_graph_replay_equals_eager_at_full_size():
+    # the bench's configuration: the 42-layer Flash backbone (2 full, 26
+    # compressed, 14 full layers) at full width on 6x34x60, 3 evaluations,
+    # captured once into a CUDA graph; the replay must reproduce the eager
+    # pass bit for bit, stay finite and move video and audio latents
+    w = S.WORKLOADS["flash_backbone_6x34x60"]
+    layers, io = S.make_weights(w, device=DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights(l) for l in layers], api.IOWeights(io), w.compress)
+    seq = api.Sequence.from_workload(w, S.pack_tokens(w), DEV)
+    inp = S.make_inputs(w, device=DEV)
+    v0, a0 = inp["video_lat"], inp["audio_lat"]
+    ve, ae = v0.clone(), a0.clone()
+    bb.sample(seq, w.video_clock, w.audio_clock, ve, inp["text_emb"], ae)
+    vg, ag = v0.clone(), a0.clone()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        bb.sample(seq, w.video_clock, w.audio_clock, vg, inp["text_emb"], ag)
+    vg.copy_(v0)
+    ag.copy_(a0)
+    graph.replay()
+    torch.cuda.synchronize()
+    del graph
+    assert torch.equal(ve, vg) and torch.equal(ae, ag)
+    assert torch.isfinite(ve).all() and torch.isfinite(ae).all()
+    assert float((ve - v0).abs().max()) > 0 and float((ae - a0).abs().max()) > 0
