@@ -31,6 +31,11 @@ Readings where the pages leave a step open:
   no integer stride).  The head's output columns are ordered
   (channel, dt, dy, dx) with dx fastest.
 * Output layout: pixels [F, c_pix, H*ps, W*ps] (frames of channel planes).
+* Colour conversion ([PaperDaily] section 二: the fully accelerated
+  configuration converts colours on the GPU): the decoder's values are read
+  as lying in [-1, 1] and mapped linearly onto 8-bit codes, 127.5 * (v + 1)
+  taken in fp32 as a product and then a sum (each rounded), clamped to
+  [0, 255] and rounded to the nearest integer, ties to even.
 """
 
 import numpy as np
@@ -89,3 +94,13 @@ def decoder_forward(latents, layers, io, T, H, W, heads, head_dim, c_pix, pt, ps
     pixels [1 + pt*(T-1), c_pix, H*ps, W*ps]."""
     x = decoder_tokens(latents, layers, io, T, H, W, heads, head_dim, rope_split, eps, theta, block_fn)
     return unpatchify(pixel_head(x, io, eps), T, H, W, c_pix, pt, ps)
+
+
+def to_rgb8(pixels):
+    """8-bit codes of decoder values (fp32 arithmetic, see the module
+    docstring): uint8 array of the same shape."""
+    v = np.asarray(pixels, dtype=np.float32)
+    t = (v * np.float32(127.5)).astype(np.float32)
+    t = (t + np.float32(127.5)).astype(np.float32)
+    t = np.clip(t, np.float32(0.0), np.float32(255.0))
+    return np.rint(t).astype(np.uint8)

@@ -146,3 +146,31 @@ def test_full_clip_shapes():
     assert (34 * 16, 60 * 16) == (544, 960)
     y = np.zeros((6 * 2 * 3, 3 * 4 * 16 * 16))
     assert D.unpatchify(y, 6, 2, 3, 3, 4, 16).shape == (21, 3, 32, 48)
+
+
+def test_rgb8_closed_form_values():
+    v = np.array([-1.0, 1.0, 0.0, -2.0, 3.0, np.float32(1 / 127.5 - 1), -1 + 3 / 127.5], dtype=np.float32)
+    # -1 -> 0, 1 -> 255, 0 -> 127.5 -> 128 (tie to even), out of range clamps,
+    # one code step above -1 -> 1, three steps -> 3
+    np.testing.assert_array_equal(D.to_rgb8(v), [0, 255, 128, 0, 255, 1, 3])
+
+
+def test_rgb8_ties_go_to_even_codes():
+    # v = (k + 0.5) / 127.5 - 1 lands (in fp32) exactly on k + 0.5 only where
+    # that is representable after the two roundings; check those cases
+    k = np.arange(0, 255)
+    v = ((k + 0.5) / 127.5 - 1).astype(np.float32)
+    t = (v * np.float32(127.5)).astype(np.float32) + np.float32(127.5)
+    exact = t.astype(np.float64) == k + 0.5
+    assert exact.sum() > 50
+    got = D.to_rgb8(v)[exact].astype(int)
+    want = np.where(k[exact] % 2 == 0, k[exact], k[exact] + 1)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_rgb8_is_monotone_and_within_half_a_code_of_the_exact_map():
+    v = np.linspace(-1.2, 1.2, 200001).astype(np.float32)
+    q = D.to_rgb8(v).astype(int)
+    assert (np.diff(q) >= 0).all()
+    exact = np.clip(127.5 * (v.astype(np.float64) + 1), 0, 255)
+    assert (np.abs(q - exact) <= 0.5 + 1e-4).all()
