@@ -452,13 +452,16 @@ class Decoder:
         T, H, W = grid
         return L.load().fsdit_decoder_workspace_size(C.byref(self.dims), C.byref(self.io.struct), T, H, W)
 
-    def forward(self, latents, grid, pixels=None, stream=None):
+    def forward(self, latents, grid, pixels=None, rgb8=False, stream=None):
+        """Pixels as fp32 values, or (rgb8) as the uint8 codes of the fused
+        colour conversion."""
         T, H, W = grid
         s = self.io.struct
         if pixels is None:
-            pixels = torch.empty(self.frames(T), s.c_pix, H * s.patch_s, W * s.patch_s, dtype=torch.float32,
-                                 device=latents.device)
+            pixels = torch.empty(self.frames(T), s.c_pix, H * s.patch_s, W * s.patch_s,
+                                 dtype=torch.uint8 if rgb8 else torch.float32, device=latents.device)
         ws = workspace(self.workspace_bytes(grid), latents.device)
         L.call("fsdit_decoder_forward", C.byref(self.dims), self.n_layers, self.layer_structs, C.byref(s), T, H, W,
-               L.ptr(latents), L.ptr(pixels), L.ptr(ws), ws.numel(), _stream(stream))
+               L.ptr(latents), L.ptr(pixels), L.PIXELS_RGB8 if rgb8 else L.PIXELS_F32, L.ptr(ws), ws.numel(),
+               _stream(stream))
         return pixels

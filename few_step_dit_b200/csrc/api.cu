@@ -182,6 +182,7 @@ static EpiParams make_ep(const fsdit_dims* d, int epi, const void* bias, void* o
   e.row_scale = nullptr;
   e.col_scale = nullptr;
   e.up_h = e.up_w = e.up_c = e.up_pt = e.up_ps = 1;
+  e.up_rgb8 = 0;
   e.split_part = nullptr;
   e.split_cnt = nullptr;
   return e;
@@ -193,8 +194,9 @@ fsdit_status launch_linear(const fsdit_dims* d, const void* a, const void* w, co
   static const int cls_of[6] = {PC_GEMM_BIAS, PC_GEMM_BIAS_F32, PC_GEMM_QKV, PC_GEMM_GELU, PC_GEMM_RESID,
                                 PC_PIXEL_HEAD};
   const double s = (double)dsize(d->dtype);
-  const double out_b =
-      (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32 || ep.epi == EPI_UNPATCH) ? 4.0 : s;
+  const double out_b = ep.epi == EPI_UNPATCH ? (ep.up_rgb8 ? 1.0 : 4.0)
+                      : (ep.epi == FSDIT_EPI_RESIDUAL || ep.epi == FSDIT_EPI_BIAS_F32) ? 4.0
+                                                                                        : s;
   const double by = ((double)M * K + (double)N * K) * s + (double)M * N * out_b +
                     (ep.epi == FSDIT_EPI_RESIDUAL ? (double)M * N * 4.0 : 0.0);
   ProfScope ps(prof_cls >= 0 ? prof_cls : cls_of[ep.epi], 1, 2.0 * M * N * K, by, st);

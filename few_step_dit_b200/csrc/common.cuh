@@ -70,6 +70,7 @@ struct EpiParams {
   const float* col_scale;  // row_scale[row] * col_scale[col] (FP8 dequantization) before the bias
   int up_h, up_w;          // EPI_UNPATCH: the rows are the cells of a (t, h, w) grid up_h x up_w per frame,
   int up_c, up_pt, up_ps;  // each column a pixel of the cell's up_c x up_pt x up_ps x up_ps patch
+  int up_rgb8;             // EPI_UNPATCH: 1 = write 8-bit codes (rgb8_code) instead of fp32 values
   float* split_part;       // pair GEMM tail cut: caller scratch for the partial accumulators
   int* split_cnt;          // (SPLIT_WS_BYTES) and its zeroed counters (SPLIT_CNT_BYTES), or null: no cut
 };
@@ -85,6 +86,14 @@ constexpr size_t SPLIT_CNT_BYTES = 64 * 16 * 4;
 // pt*t + dt - (pt - 1) (dropped when negative: latent frame 0 yields one
 // frame), pixel (ps*h + dy, ps*w + dx).
 constexpr int EPI_UNPATCH = 5;
+
+// Colour conversion of a decoder value to its 8-bit code: 127.5 * (v + 1) as
+// a rounded product and a rounded sum in fp32, clamped to [0, 255], rounded
+// to the nearest integer (ties to even).
+__device__ __forceinline__ uint32_t rgb8_code(float v) {
+  const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(v, 127.5f), 127.5f), 0.0f), 255.0f);
+  return (uint32_t)__float2int_rn(t);
+}
 
 // Element offset of column `col` of row `row` in the frames, -1 if dropped.
 __device__ __forceinline__ long long unpatch_offset(const EpiParams& p, int row, int col) {
@@ -138,11 +147,12 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
     for (int i = 0; i < CNT; ++i) v[i] = gelu_tanh(v[i]);
   }
   if (p.epi == EPI_UNPATCH) {
-    float* o = reinterpret_cast<float*>(p.out);
 #pragma unroll
     for (int i = 0; i < CNT; ++i) {
       const long long off = unpatch_offset(p, row, col + i);
-      if (off >= 0) o[off] = v[i];
+      if (off < 0) continue;
+      if (p.up_rgb8) reinterpret_cast<uint8_t*>(p.out)[off] = (uint8_t)rgb8_code(v[i]);
+      else reinterpret_cast<float*>(p.out)[off] = v[i];
     }
   } else if (p.epi == FSDIT_EPI_RESIDUAL) {
     const float* r = p.resid + (size_t)row * p.ldr + col;
@@ -287,13 +297,18 @@ __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col
   }
   if (p.epi == EPI_UNPATCH) {
     // up_ps % 4 == 0: each group of 4 columns is 4 adjacent pixels of one
-    // pixel row, 16-byte aligned in the frames
-    float* o = reinterpret_cast<float*>(p.out);
+    // pixel row, 16-byte aligned in fp32 frames, 4-byte aligned in 8-bit ones
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const long long off = unpatch_offset(p, row, col + 4 * i);
-      if (off >= 0)
-        *reinterpret_cast<float4*>(o + off) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if (off < 0) continue;
+      if (p.up_rgb8)
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.out) + off) =
+            rgb8_code(v[4 * i]) | (rgb8_code(v[4 * i + 1]) << 8) | (rgb8_code(v[4 * i + 2]) << 16) |
+            (rgb8_code(v[4 * i + 3]) << 24);
+      else
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + off) =
+            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
   } else if (p.epi == FSDIT_EPI_RESIDUAL) {
     float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col);

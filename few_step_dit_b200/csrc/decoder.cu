@@ -6,7 +6,9 @@
 //   at full resolution (the same block body, GEMMs and attention as the
 //   denoiser) -> final RMSNorm -> pixel head on the tensor cores whose
 //   epilogue writes every value straight to its frame, channel and pixel
-//   (EPI_UNPATCH: no [cells, patch] intermediate and no permute pass).
+//   (EPI_UNPATCH: no [cells, patch] intermediate and no permute pass), as
+//   fp32 or, with the GPU-side colour conversion of [PaperDaily] section 二,
+//   as 8-bit codes.
 // Included by libfsdit.cu after api.cu, whose block helpers it reuses.
 
 namespace fsdit {
@@ -84,7 +86,8 @@ size_t fsdit_decoder_workspace_size(const fsdit_dims* dims, const fsdit_decoder_
 
 fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
                                    const fsdit_decoder_io* io, int T, int H, int W, const float* latents,
-                                   float* pixels, void* workspace, size_t ws_bytes, fsdit_stream_t stream) {
+                                   void* pixels, int pixel_format, void* workspace, size_t ws_bytes,
+                                   fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));
   FS_TRY(check_decoder_io(io));
   FS_TRY(check_decoder_grid(T, H, W));
@@ -93,6 +96,10 @@ fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const f
     return FSDIT_E_NULL;
   }
   for (int l = 0; l < n_layers; ++l) FS_TRY(check_block_weights(dims, &layers[l]));
+  if (pixel_format != FSDIT_PIXELS_F32 && pixel_format != FSDIT_PIXELS_RGB8) {
+    set_error("decoder: pixel_format %d is neither FSDIT_PIXELS_F32 nor FSDIT_PIXELS_RGB8", pixel_format);
+    return FSDIT_E_DTYPE;
+  }
   FS_TRY(need(latents, "latents"));
   FS_TRY(need(pixels, "pixels"));
   FS_TRY(need(workspace, "workspace"));
@@ -124,6 +131,7 @@ fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const f
   ep.up_c = io->c_pix;
   ep.up_pt = io->patch_t;
   ep.up_ps = io->patch_s;
+  ep.up_rgb8 = pixel_format == FSDIT_PIXELS_RGB8 ? 1 : 0;
   return launch_linear(dims, ws.xn, io->w_out, ep, N, n_out, Hd, st, PC_PIXEL_HEAD);
 }
 

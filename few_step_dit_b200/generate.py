@@ -11,9 +11,10 @@ Long video (--chunks N): chunk after chunk with the bounded history store; every
 chunk after the first starts from the previous chunk's last latent frame (its
 boundary), is decoded on its own and loses the boundary's frame, so the clip
 grows by 4 x (T - 1) frames a chunk.  Frames are written as uint8 RGB
-[frames, 3, height, width] (values mapped from [-1, 1]).  No trained weights are
-available, so the frames are noise-like: the command exercises and times the
-path (one JSON line with the stage times on stdout).
+[frames, 3, height, width]: the decoder's pixel head converts its values from
+[-1, 1] to 8-bit codes on the GPU (fsdit_decoder_forward, FSDIT_PIXELS_RGB8).
+No trained weights are available, so the frames are noise-like: the command
+exercises and times the path (one JSON line with the stage times on stdout).
 """
 
 from __future__ import annotations
@@ -42,10 +43,6 @@ def tiny_workloads():
     wd = S.scaled(S.DECODER_WORKLOADS["decoder_6x34x60"], hidden=256, heads=2, ffn=1024, n_layers=2,
                   grid=(3, 6, 8), patch_s=4)
     return wb, wd
-
-
-def to_uint8(frames):
-    return ((frames.clamp(-1.0, 1.0) + 1.0) * 127.5).round().to(torch.uint8)
 
 
 def run(backbone="flash_backbone_6x34x60", proj_fp8=False, chunks=0, tiny=False, seed=S.SEED_INPUTS,
@@ -83,11 +80,11 @@ def run(backbone="flash_backbone_6x34x60", proj_fp8=False, chunks=0, tiny=False,
         e0.record()
         bb.sample(seq, wb.video_clock, wb.audio_clock, vl, inp["text_emb"], al)
         e1.record()
-        px = dec.forward(vl[:wb.n_video], wd.grid)
+        px = dec.forward(vl[:wb.n_video], wd.grid, rgb8=True)
         e2.record()
         e2.synchronize()
         t_sample, t_decode = e0.elapsed_time(e1), e1.elapsed_time(e2)
-        out.append(to_uint8(px).cpu())
+        out.append(px.cpu())
     else:
         lv = api.LongVideo(bb, wb.grid, wb.n_text, wb.n_audio, wb.video_ch, device=device)
         for k in range(chunks):
@@ -97,12 +94,12 @@ def run(backbone="flash_backbone_6x34x60", proj_fp8=False, chunks=0, tiny=False,
             e0.record()
             lat, _ = lv.chunk(noise_v, text, noise_a, wb.video_clock, wb.audio_clock)
             e1.record()
-            px = dec.forward(lat, wd.grid)
+            px = dec.forward(lat, wd.grid, rgb8=True)
             e2.record()
             e2.synchronize()
             t_sample += e0.elapsed_time(e1)
             t_decode += e1.elapsed_time(e2)
-            out.append(to_uint8(px if k == 0 else px[1:]).cpu())  # drop the boundary's frame
+            out.append((px if k == 0 else px[1:]).cpu())  # drop the boundary's frame
     api.device_error()
     frames = torch.cat(out)
     return frames, {"sample_ms": t_sample, "decode_ms": t_decode}

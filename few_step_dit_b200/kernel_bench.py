@@ -231,12 +231,13 @@ def case_decoder(a):
     CUDA graph; plus a per-kernel-class profile of one eager run."""
     w, dec = _decoder(a)
     lat = S.make_decoder_latents(w, device="cuda")
-    px = torch.empty(w.pixel_shape, device="cuda")
-    step = lambda: dec.forward(lat, w.grid, pixels=px)  # noqa: E731
+    px = torch.empty(w.pixel_shape, dtype=torch.uint8 if a.rgb8 else torch.float32, device="cuda")
+    step = lambda: dec.forward(lat, w.grid, pixels=px, rgb8=a.rgb8)  # noqa: E731
     ms = _graph_ms(step, a)
     tflop = _decoder_flops(w) / 1e12
     T, H, W = w.grid
-    return {"case": "decoder", "workload": f"decoder_{T}x{H}x{W}", "fp8": bool(a.fp8), "cells": w.n_cells,
+    return {"case": "decoder", "workload": f"decoder_{T}x{H}x{W}", "fp8": bool(a.fp8), "rgb8": bool(a.rgb8),
+            "cells": w.n_cells,
             "frames": w.n_frames, "ms": ms, "tflop": tflop, "tflops": tflop / ms * 1e3,
             "frames_per_s": w.n_frames / ms * 1e3, "classes": _profile(step)}
 
@@ -291,6 +292,7 @@ def main():
     p.add_argument("--grid", default="", help="chunk / decoder: latent grid TxHxW (default 6x34x60)")
     p.add_argument("--cut", action="store_true", help="gemm: cut the last wave's tiles along K (fsdit_linear_ws)")
     p.add_argument("--backbone", default="flash_backbone_6x34x60", help="generate: the backbone workload")
+    p.add_argument("--rgb8", action="store_true", help="decoder: 8-bit RGB frames (fused colour conversion)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()

@@ -71,6 +71,7 @@ HISTORY_MAX_ENTRIES = 11
 HISTORY_MIN_SLOTS = 12
 
 DECODER_IO_FIELDS = ("w_in", "b_in", "g_out", "w_out", "b_out")
+PIXELS_F32, PIXELS_RGB8 = 0, 1
 
 
 class DecoderIO(C.Structure):
@@ -131,7 +132,7 @@ _SIGS = {
     "fsdit_decoder_frames": (_I, [_I, _I]),
     "fsdit_decoder_workspace_size": (C.c_size_t, [C.POINTER(Dims), C.POINTER(DecoderIO), _I, _I, _I]),
     "fsdit_decoder_forward": (_I, [C.POINTER(Dims), _I, C.POINTER(BlockWeights), C.POINTER(DecoderIO), _I, _I,
-                                   _I, _P, _P, _P, C.c_size_t, _P]),
+                                   _I, _P, _P, _I, _P, C.c_size_t, _P]),
 }
 
 _lib = None

@@ -503,18 +503,27 @@ FSDIT_API int fsdit_decoder_frames(int T, int patch_t);
 FSDIT_API size_t fsdit_decoder_workspace_size(const fsdit_dims* dims, const fsdit_decoder_io* io, int T, int H,
                                               int W);
 
+/* Pixel formats of fsdit_decoder_forward.  FSDIT_PIXELS_RGB8 is the GPU-side
+ * colour conversion of [PaperDaily] section 二 (the fully accelerated
+ * configuration), fused into the pixel head: each value v, read as lying in
+ * [-1, 1], becomes the code round_half_even(clamp(127.5 * (v + 1), 0, 255)),
+ * the product and the sum each rounded to fp32. */
+enum { FSDIT_PIXELS_F32 = 0, FSDIT_PIXELS_RGB8 = 1 };
+
 /* Decode latents (device, fp32 [T*H*W][c_lat], cells (t, h, w) row-major) into
- * pixels (device, fp32 [fsdit_decoder_frames(T, patch_t)][c_pix][H*patch_s]
- * [W*patch_s], 16-byte aligned, fully written).  layers: host array of
+ * pixels (device, [fsdit_decoder_frames(T, patch_t)][c_pix][H*patch_s]
+ * [W*patch_s] of fp32 values or uint8 codes per pixel_format, 16-byte aligned,
+ * fully written).  layers: host array of
  * n_layers block weights (device pointers; with dims.proj_fp8 the E4M3 weights
  * and scales as for the backbone).  The residual stream is fp32; the GEMMs and
  * attention run as in the backbone (bf16 on the tcgen05 tensor cores, or
  * exact fp32 with dims.dtype FSDIT_F32).  Errors: FSDIT_E_NULL,
  * FSDIT_E_SHAPE (grid empty, c_lat outside 1..64, patch sizes not positive,
- * patch_s % 4 != 0), FSDIT_E_ALIGN, FSDIT_E_WORKSPACE. */
+ * patch_s % 4 != 0), FSDIT_E_DTYPE (unknown pixel_format), FSDIT_E_ALIGN,
+ * FSDIT_E_WORKSPACE. */
 FSDIT_API fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const fsdit_block_weights* layers,
                                              const fsdit_decoder_io* io, int T, int H, int W, const float* latents,
-                                             float* pixels, void* workspace, size_t ws_bytes,
+                                             void* pixels, int pixel_format, void* workspace, size_t ws_bytes,
                                              fsdit_stream_t stream);
 
 #ifdef __cplusplus

@@ -130,12 +130,15 @@ def test_decoder_forward_rejects_bad_arguments_without_launching(fs):
     w = (L.BlockWeights * 1)(L.BlockWeights(*([0x10000] * 10)))
     big = 1 << 40
     f = fs.fsdit_decoder_forward
-    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, None, fake, fake, big, None) == -1
-    assert f(C.byref(d), 1, None, C.byref(_dec_io()), 6, 34, 60, fake, fake, fake, big, None) == -1
-    assert f(C.byref(d), 1, w, C.byref(_dec_io(patch_s=2)), 6, 34, 60, fake, fake, fake, big, None) == -2
-    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 0, 60, fake, fake, fake, big, None) == -2
-    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, odd, fake, big, None) == -3
-    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, fake, fake, 1024, None) == -6
+    rgb = L.PIXELS_RGB8
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, None, fake, 0, fake, big, None) == -1
+    assert f(C.byref(d), 1, None, C.byref(_dec_io()), 6, 34, 60, fake, fake, 0, fake, big, None) == -1
+    assert f(C.byref(d), 1, w, C.byref(_dec_io(patch_s=2)), 6, 34, 60, fake, fake, 0, fake, big, None) == -2
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 0, 60, fake, fake, 0, fake, big, None) == -2
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, odd, rgb, fake, big, None) == -3
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, fake, 2, fake, big, None) == -4
+    assert "pixel_format" in L.last_error()
+    assert f(C.byref(d), 1, w, C.byref(_dec_io()), 6, 34, 60, fake, fake, rgb, fake, 1024, None) == -6
     assert "workspace" in L.last_error()
 
 

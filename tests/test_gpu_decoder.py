@@ -91,6 +91,26 @@ def test_fp8_decoder_matches_fp8_oracle():
     assert O.rel_l2(got, ref) < 3e-2
 
 
+@pytest.mark.parametrize("kw", [{}, {"dtype": "bf16", "grid": (3, 9, 10), "patch_s": 16},
+                                {"dtype": "bf16", "grid": (2, 7, 11), "patch_s": 4, "c_pix": 1, "patch_t": 1}])
+def test_rgb8_frames_are_the_colour_conversion_of_the_fp32_frames(kw):
+    # the fused colour conversion decides every code in fp32 from the same
+    # values the fp32 output holds, so the codes are bit-exact against the
+    # oracle's conversion of those values
+    w = S.scaled(TINY, **kw)
+    layers, io = S.make_decoder_weights(w)
+    lat = S.make_decoder_latents(w).to(DEV)
+    dec = api.Decoder(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.DecoderIO({k: v.to(DEV) for k, v in io.items()}, w.c_pix, w.patch_t, w.patch_s))
+    f32 = dec.forward(lat, w.grid)
+    u8 = dec.forward(lat, w.grid, rgb8=True)
+    torch.cuda.synchronize()
+    assert u8.dtype == torch.uint8 and tuple(u8.shape) == w.pixel_shape
+    want = D.to_rgb8(f32.cpu().numpy())
+    np.testing.assert_array_equal(u8.cpu().numpy(), want)
+    assert 0 < want.mean() < 255
+
+
 FULL = S.DECODER_WORKLOADS["decoder_6x34x60"]
 
 
@@ -145,6 +165,16 @@ def test_full_clip_sampled_cells(full_weights, n_layers):
     got = np.concatenate([_cell_pixels(FULL, px, int(c)).ravel() for c in cells])
     ref = np.concatenate([_oracle_cell_pixels(FULL, y[i], int(c)).ravel() for i, c in enumerate(cells)])
     assert O.rel_l2(got, ref) < 1e-2
+
+
+def test_full_clip_rgb8_codes(full_weights):
+    (layers, io), lat = full_weights
+    dec = _full_decoder(layers, io, 1)
+    f32 = dec.forward(lat, FULL.grid)
+    u8 = torch.full(FULL.pixel_shape, 7, dtype=torch.uint8, device=DEV)
+    dec.forward(lat, FULL.grid, pixels=u8, rgb8=True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(u8.cpu().numpy(), D.to_rgb8(f32.cpu().numpy()))
 
 
 def test_full_26_layer_decoder_writes_every_pixel():
