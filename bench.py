@@ -16,6 +16,7 @@ the fp64 CPU oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -301,6 +302,8 @@ def run_fsdit(args, rank, world, local_rank):
         al.copy_(al0)
         bb.sample(seq, w.video_clock, w.audio_clock, vl, text, al, compress=compress)
 
+    gc.collect()
+    torch.cuda.reset_peak_memory_stats(device)  # setup copies (e.g. weights before quantizing) do not count
     for _ in range(args.warmup):
         step()
     api.device_error()
@@ -415,6 +418,9 @@ def run_fsdit(args, rank, world, local_rank):
         line["compression_speedup"] = full_ms / ms_per_step
     if clk is not None:
         line["clocks"] = clk
+    # peak device memory of the warm-up, timed and comparison passes: every
+    # device buffer (weights, latents, workspaces) is a torch allocation
+    line["peak_mem_gb"] = round(torch.cuda.max_memory_allocated(device) / 1e9, 2)
     if args.proj_fp8:
         line["tensor_peak_basis"] = "bf16 sustained peak (attention still runs in bf16)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.proj_fp8:
