@@ -244,7 +244,12 @@ _ws_cache: dict = {}
 
 
 def workspace(nbytes, device):
-    """A cached uint8 device buffer of at least nbytes (caller-side allocation)."""
+    """A cached uint8 device buffer of at least nbytes (caller-side allocation).
+
+    One buffer per device serves every call of this module, so calls on one
+    device must not overlap in time (issue them on one stream, or synchronize
+    between streams); concurrent work needs the C ABI with a workspace per
+    stream."""
     key = str(device)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
