@@ -9,3 +9,4 @@
 #include "noalloc.cu"
 #include "history.cu"
 #include "decoder.cu"
+#include "selfcheck.cu"

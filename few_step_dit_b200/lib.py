@@ -125,6 +125,7 @@ _SIGS = {
     "fsdit_history_gather": (_I, [C.POINTER(HistoryStore), C.POINTER(HistoryEntry), _I, _P, _I, _P, _P]),
     "fsdit_history_copy_frame": (_I, [C.POINTER(HistoryStore), _I, _P, _P]),
     "fsdit_chunk_tags": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "fsdit_check_bounded_wait": (_I, [_P, _P]),
     "fsdit_gemm_scratch_size": (C.c_size_t, []),
     "fsdit_linear_ws": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, C.c_size_t, _P]),
     "fsdit_linear_fp8_ws": (_I, [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, C.c_size_t,

@@ -147,6 +147,15 @@ FSDIT_API const char* fsdit_version(void);
  * reset gave up a bounded wait (and clears the word), else FSDIT_OK. */
 FSDIT_API fsdit_status fsdit_device_error(fsdit_stream_t stream);
 
+/* Failure-path check (no fault): launches one thread that waits, through the
+ * bounded mbarrier wait every tensor-core kernel of the library uses, on a
+ * barrier nothing arrives at.  The wait gives up after its limit (~2 s of SM
+ * clocks), sets the device error word and returns; result (device, int[2])
+ * receives {wait completed (0), abort flag set (1)}.  A following
+ * fsdit_device_error() returns FSDIT_E_TIMEOUT (and clears the word); the
+ * context stays usable. */
+FSDIT_API fsdit_status fsdit_check_bounded_wait(int* result, fsdit_stream_t stream);
+
 /* Launch profiler (measurement aid, off by default).  Between
  * fsdit_profile_start(max_launches) and fsdit_profile_stop() every launch the
  * library enqueues is bracketed by a CUDA event pair on its own stream (events
