@@ -1,7 +1,8 @@
 """Full-size parity: the full-width Flash block on the 6x34x60 grid (12,560
-tokens, hidden 5376, 56 heads, FFN 14336, bf16) in the launch configuration the
-bench uses, checked on sampled output rows that the oracle computes one by one
-(relative L2 <= 1e-2 on the rows and on their update y - x); plus the
+tokens, hidden 5376, 56 heads, FFN 14336, bf16) and on the compression sweep's
+6x17x30 and 12x34x60 grids, in the launch configuration the bench uses, checked
+on sampled output rows that the oracle computes one by one (relative L2 <= 1e-2
+on the rows and on their update y - x); plus the
 standard model's control-frame packing through the stack and the 4-evaluation
 sampler at small width."""
 
@@ -44,9 +45,7 @@ def _sample_rows(w, seed=11):
     return np.unique(np.concatenate([fixed, rng.integers(0, N, 32)]))
 
 
-@pytest.mark.parametrize("compress", [True, False])
-def test_full_width_block_sampled_rows(full_block, compress):
-    w, wts, x, tags = full_block
+def _sampled_rows_case(w, wts, x, tags, compress):
     dims = api.dims_of(w)
     seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
     bw = api.BlockWeights({k: v.to(DEV) for k, v in wts.items()})
@@ -63,6 +62,22 @@ def test_full_width_block_sampled_rows(full_block, compress):
         ref = O.dit_block_rows(xn, wn, tags["pos"], w.heads, w.head_dim, rows)
     assert O.rel_l2(got, ref) < 1e-2
     assert O.rel_l2(got - xn[rows], ref - xn[rows]) < 1e-2
+
+
+@pytest.mark.parametrize("compress", [True, False])
+def test_full_width_block_sampled_rows(full_block, compress):
+    _sampled_rows_case(*full_block, compress)
+
+
+@pytest.mark.parametrize("grid", [(6, 17, 30), (12, 34, 60)])
+@pytest.mark.parametrize("compress", [True, False])
+def test_sweep_grids_full_width_block_sampled_rows(grid, compress):
+    # the compression sweep's other grids (3,060 and 24,480 video tokens, 864
+    # and 6,696 kept) with the same full-width block
+    w = S.WORKLOADS["flash_block_%dx%dx%d" % grid]
+    layers, _ = S.make_weights(w, n_layers=1)
+    inp = S.make_inputs(w)
+    _sampled_rows_case(w, layers[0], inp["x"].float(), S.pack_tokens(w), compress)
 
 
 def test_full_width_block_properties_at_every_row(full_block):
