@@ -302,10 +302,12 @@ def dit_block_compressed(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video
 
 
 def dit_block_compressed_rows(x, w, pos, heads, head_dim, keep_idx, near_idx, n_video, rows,
-                              rope_split=(32, 48, 48), eps=1e-6, theta=10000.0):
+                              rope_split=(32, 48, 48), eps=1e-6, theta=10000.0, rows_fn=None):
     """``dit_block_compressed(...)[rows]`` for the requested rows only: the
-    compressed block is evaluated (via ``dit_block_rows``) just for the
+    compressed block is evaluated (via ``dit_block_rows``, or ``rows_fn`` with
+    the same signature, e.g. the low-bit block's row restriction) just for the
     compressed rows those outputs read, then the same broadcast rule applies."""
+    rows_fn = rows_fn or dit_block_rows
     x = np.asarray(x, dtype=F64)
     rows = np.asarray(rows, dtype=np.int64)
     keep_idx = np.asarray(keep_idx, dtype=np.int64)
@@ -316,7 +318,7 @@ def dit_block_compressed_rows(x, w, pos, heads, head_dim, keep_idx, near_idx, n_
     x_c = gather_rows(x, keep_idx, n_video)
     pos_c = gather_rows(pos, keep_idx, n_video)
     y_c = np.zeros_like(x_c)
-    y_c[need] = dit_block_rows(x_c, w, pos_c, heads, head_dim, need, rope_split, eps, theta)
+    y_c[need] = rows_fn(x_c, w, pos_c, heads, head_dim, need, rope_split, eps, theta)
     return broadcast_residual(x, y_c, keep_idx, near_idx, n_video)[rows]
 
 

@@ -110,3 +110,33 @@ def dit_block_fp8(x, w, pos, heads, head_dim, rope_split=(32, 48, 48), eps=1e-6,
     u = gelu_tanh(linear_fp8(qh, sh, *wq["w_1"], w["b_1"]))
     qu, su = quantize_rows(bf16_round(u).astype(F32))
     return h + linear_fp8(qu, su, *wq["w_2"], w["b_2"])
+
+
+def dit_block_fp8_rows(x, w, pos, heads, head_dim, rows, rope_split=(32, 48, 48), eps=1e-6, theta=10000.0,
+                       wq=None):
+    """``dit_block_fp8(x, ...)[rows]`` for the requested rows only.  Every
+    row's normalized input is quantized (its own scale) and projected to keys
+    and values; queries, the output projection and the FFN only for ``rows``.
+    Each quantization depends on its own row alone, so the restriction is
+    exact -- used to check full-size E4M3 blocks one row at a time."""
+    x = np.asarray(x, dtype=F64)
+    rows = np.asarray(rows, dtype=np.int64)
+    if wq is None:
+        wq = quantize_block_weights(w)
+    A = heads * head_dim
+    n, r = x.shape[0], len(rows)
+    qa, sa = quantize_rows(rms_norm(x, w["g_attn"], eps).astype(F32))
+    qw, sw = wq["w_qkv"]
+    b = np.asarray(w["b_qkv"], dtype=F64)
+    q = linear_fp8(qa[rows], sa[rows], qw[:A], sw[:A], b[:A]).reshape(r, heads, head_dim)
+    k = linear_fp8(qa, sa, qw[A:2 * A], sw[A:2 * A], b[A:2 * A]).reshape(n, heads, head_dim)
+    v = linear_fp8(qa, sa, qw[2 * A:], sw[2 * A:], b[2 * A:]).reshape(n, heads, head_dim)
+    q = apply_rope(q, np.asarray(pos)[rows], rope_split, theta)
+    k = apply_rope(k, pos, rope_split, theta)
+    o = attention(q, k, v)
+    qo, so = quantize_rows(bf16_round(o).astype(F32))
+    h = x[rows] + linear_fp8(qo, so, *wq["w_o"], w["b_o"])
+    qh, sh = quantize_rows(rms_norm(h, w["g_ffn"], eps).astype(F32))
+    u = gelu_tanh(linear_fp8(qh, sh, *wq["w_1"], w["b_1"]))
+    qu, su = quantize_rows(bf16_round(u).astype(F32))
+    return h + linear_fp8(qu, su, *wq["w_2"], w["b_2"])

@@ -140,3 +140,22 @@ def test_fp8_block_decisions_use_fp32_inputs():
     q2, s2 = Q.quantize_rows((xn * (1 + 1e-12)).astype(np.float32))
     np.testing.assert_array_equal(q1, q2)
     np.testing.assert_array_equal(s1, s2)
+
+
+def test_fp8_block_row_restriction_equals_the_block():
+    # the row-restricted E4M3 block reproduces the full block's rows (each
+    # quantization depends on its own row), also through the compressed form
+    rng = np.random.default_rng(12)
+    n = 40
+    w = _tiny(rng)
+    x = rng.standard_normal((n, 256)).astype(np.float32).astype(np.float64)
+    pos = rng.integers(0, 9, (n, 3))
+    rows = np.array([0, 3, 17, 39])
+    full = Q.dit_block_fp8(x, w, pos, 2, 128)
+    np.testing.assert_allclose(Q.dit_block_fp8_rows(x, w, pos, 2, 128, rows), full[rows], rtol=1e-10, atol=1e-12)
+    # compressed: a 2 x 4 x 5 grid (40 rows, no text/audio)
+    k, nn = O.keep_map(2, 4, 5)
+    pos_g = np.stack(np.meshgrid(np.arange(2), np.arange(4), np.arange(5), indexing="ij"), -1).reshape(-1, 3)
+    fullc = O.dit_block_compressed(x, w, pos_g, 2, 128, k, nn, n, block_fn=Q.dit_block_fp8)
+    got = O.dit_block_compressed_rows(x, w, pos_g, 2, 128, k, nn, n, rows, rows_fn=Q.dit_block_fp8_rows)
+    np.testing.assert_allclose(got, fullc[rows], rtol=1e-10, atol=1e-12)
