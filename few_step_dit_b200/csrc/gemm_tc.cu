@@ -202,13 +202,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 // 128 of the 256 B rows per K step, which halves the B operand's
 // shared-memory and L2 traffic per FLOP.  A stage holds two 128-byte-wide
 // boxes of each operand (64 KB per CTA, 3 stages): eight MMAs per barrier
-// round trip.  Roles per CTA as above; warp 1 of
+// round trip.  Roles per CTA as above, but with eight epilogue warps (320
+// threads: two per TMEM lane quarter, each on half the columns); warp 1 of
 // CTA rank 0 issues the pair MMAs.  Both CTAs' TMA copies of a stage complete
 // on rank 0's `full` barrier (rank 0 expects the bytes of both); the MMA
 // commits release the stage in both CTAs.  Accumulator rows 0..127 of a tile
 // sit in rank 0's TMEM, 128..255 in rank 1's; each CTA's epilogue stores its
 // own rows and releases the accumulator buffer on rank 0's barrier (one arrive
-// per warp).
+// per warp).  SPLIT = true instantiates the opt-in tail cut's second launch
+// (units of K-slices of the last wave's tiles, see split_unit_epilogue).
 namespace gemm2 {
 
 // Tail cut bounds: at most SPLIT_MAX_UNITS partial units (256 KB of fp32
