@@ -93,14 +93,20 @@ def test_fp8_decoder_matches_fp8_oracle():
 
 @pytest.mark.parametrize("kw", [{}, {"dtype": "bf16", "grid": (3, 9, 10), "patch_s": 16},
                                 {"dtype": "bf16", "grid": (2, 7, 11), "patch_s": 4, "c_pix": 1, "patch_t": 1}])
-def test_rgb8_frames_are_the_colour_conversion_of_the_fp32_frames(kw):
+@pytest.mark.parametrize("fp8", [False, True])
+def test_rgb8_frames_are_the_colour_conversion_of_the_fp32_frames(kw, fp8):
     # the fused colour conversion decides every code in fp32 from the same
     # values the fp32 output holds, so the codes are bit-exact against the
-    # oracle's conversion of those values
+    # oracle's conversion of those values (with bf16 or E4M3 block projections)
     w = S.scaled(TINY, **kw)
+    if fp8 and w.dtype != "bf16":
+        pytest.skip("E4M3 projections run on bf16 workloads")
     layers, io = S.make_decoder_weights(w)
     lat = S.make_decoder_latents(w).to(DEV)
-    dec = api.Decoder(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+    bl = [{k: v.to(DEV) for k, v in l.items()} for l in layers]
+    if fp8:
+        bl = [api.quantize_block_weights(l) for l in bl]
+    dec = api.Decoder(api.dims_of(w, proj_fp8=fp8), [api.BlockWeights(l) for l in bl],
                       api.DecoderIO({k: v.to(DEV) for k, v in io.items()}, w.c_pix, w.patch_t, w.patch_s))
     f32 = dec.forward(lat, w.grid)
     u8 = dec.forward(lat, w.grid, rgb8=True)

@@ -118,7 +118,8 @@ def test_linear_tail_cut_residual_in_place(scratch):
     assert O.rel_l2(xd.double().cpu().numpy(), ref) < 1e-4
 
 
-@pytest.mark.parametrize("M,N,K,epi", [(1000, 2048, 8192, L.EPI_RESIDUAL), (300, 512, 8192, L.EPI_BIAS)])
+@pytest.mark.parametrize("M,N,K,epi", [(1000, 2048, 8192, L.EPI_RESIDUAL), (300, 512, 8192, L.EPI_BIAS),
+                                       (300, 768, 8192, L.EPI_QKV_ROPE)])
 def test_fp8_tail_cut_on_identical_quantized_operands(scratch, M, N, K, epi):
     rng = np.random.default_rng(8)
     a = (rng.standard_normal((M, K)) * rng.uniform(0.1, 10, (M, 1))).astype(np.float32)
@@ -127,13 +128,16 @@ def test_fp8_tail_cut_on_identical_quantized_operands(scratch, M, N, K, epi):
     qw, sw = Q.quantize_rows(w)
     b = torch.tensor(rng.standard_normal(N) * 0.05).bfloat16()
     resid = rng.standard_normal((M, N)).astype(np.float32) if epi == L.EPI_RESIDUAL else None
+    pos = rng.integers(0, 40, (M, 3)).astype(np.int32) if epi == L.EPI_QKV_ROPE else None
     codes = lambda v: torch.tensor(v).to(torch.float8_e4m3fn).view(torch.uint8).to(DEV)  # noqa: E731
-    dims = api.make_dims(256, 2, 512, L.BF16, proj_fp8=True)
+    A = N // 3 if epi == L.EPI_QKV_ROPE else 256
+    dims = api.make_dims(A, A // 128, 512, L.BF16, proj_fp8=True)
     out = api.linear_fp8(dims, codes(qa), torch.tensor(sa, dtype=torch.float32).to(DEV), codes(qw),
                          torch.tensor(sw, dtype=torch.float32).to(DEV), b.to(DEV), epi,
-                         resid=torch.tensor(resid).to(DEV) if resid is not None else None, scratch=scratch)
+                         resid=torch.tensor(resid).to(DEV) if resid is not None else None,
+                         pos=torch.tensor(pos).to(DEV) if pos is not None else None, scratch=scratch)
     torch.cuda.synchronize()
     y = Q.linear_fp8(qa, sa, qw, sw, b.double().numpy())
-    ref = resid.astype(np.float64) + y if resid is not None else y
+    ref = _ref_epilogue(y, epi, resid.astype(np.float64) if resid is not None else None, pos, A)
     bound = 1e-5 if out.dtype == torch.float32 else 5e-3
     assert O.rel_l2(out.double().cpu().numpy(), ref) < bound
