@@ -118,6 +118,7 @@ def gelu_tanh(x):
 
 
 def silu(x):
+    """SiLU, x * sigmoid(x) (the timestep MLP's activation, reading R7)."""
     x = np.asarray(x, dtype=F64)
     return x / (1.0 + np.exp(-x))
 
@@ -174,6 +175,7 @@ def attention(q, k, v):
 
 
 def linear(x, w, b=None):
+    """x W^T (+ b) in float64; W in Linear layout [out, in]."""
     y = np.asarray(x, dtype=F64) @ np.asarray(w, dtype=F64).T
     if b is not None:
         y = y + np.asarray(b, dtype=F64)
