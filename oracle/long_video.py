@@ -81,6 +81,8 @@ def history_select(n_frames: int):
 
 
 def history_token_count(n_frames: int, H: int, W: int) -> int:
+    """Rows of the history of a chunk preceded by ``n_frames`` latent frames:
+    the stride-sampled positions of every frame ``history_select`` keeps."""
     return sum(len(stride_positions(H, W, s)) for _, s in history_select(n_frames))
 
 
