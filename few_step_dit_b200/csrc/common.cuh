@@ -336,6 +336,173 @@ __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col
   }
 }
 
+// ------------------------------- coalesced epilogue of a warp's 32 x 32 block
+// After tcgen05.ld lane r of a warp holds the 32 columns of row r of a 32 x 32
+// accumulator block, so every lane's bias / residual / RoPE-table / output
+// access hits a different row: one 16-byte piece per row and instruction.
+// warp_transpose32 passes the block through 4 KB of the warp's shared memory
+// (16-byte pieces, XOR-swizzled so that neither the writes nor the reads
+// conflict) so that lane l then holds columns 4*(l%8) .. 4*(l%8)+3 of rows
+// l/8 + 4i, i = 0..7: eight lanes share one row's 128 contiguous bytes and
+// each global access of the epilogue covers four rows.  The arithmetic per
+// element is that of epi32_apply, in the same order.
+__device__ __forceinline__ void warp_transpose32(float4* buf, const float* v, float* w, int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    buf[lane * 8 + (j ^ (lane & 7))] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = (lane >> 3) + 4 * i;
+    const float4 t = buf[r * 8 + ((lane & 7) ^ (r & 7))];
+    w[4 * i] = t.x;
+    w[4 * i + 1] = t.y;
+    w[4 * i + 2] = t.z;
+    w[4 * i + 3] = t.w;
+  }
+  __syncwarp();  // the block is read before the buffer is written again
+}
+
+// Per-lane inputs of the transposed block (columns cl .. cl+3 of rows r0 + 4i).
+struct EpiTPre {
+  uint2 bias;       // the 4 bf16 bias values of the lane's columns
+  float4 cscale;    // FP8 dequantization: the 4 column scales
+  float rscale[8];  //                     and the row scale of each of the 8 rows
+  float4 extra[8];  // QKV_ROPE: (cos, sin) of the lane's 2 pairs; RESIDUAL: 4 fp32 values; per row
+};
+
+// Loads for columns [col, col + 32) (all inside the output) of the block whose
+// first row is row0; rows at or past M are skipped.  Alignment as for
+// epi32_prefetch.
+__device__ __forceinline__ void epiT_prefetch(const EpiParams& p, int row0, int col, int M, int lane,
+                                              EpiTPre& e) {
+  const int cl = col + 4 * (lane & 7);
+  const int r0 = row0 + (lane >> 3);
+  e.bias = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(p.bias) + cl));
+  if (p.col_scale != nullptr) {
+    e.cscale = __ldg(reinterpret_cast<const float4*>(p.col_scale + cl));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e.rscale[i] = r0 + 4 * i < M ? __ldg(p.row_scale + r0 + 4 * i) : 0.0f;
+  }
+  if (p.epi == FSDIT_EPI_QKV_ROPE) {
+    if (col < p.rope_cols && p.rope_cs != nullptr) {
+      const int pair = (cl & (p.head_dim - 1)) >> 1;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (r0 + 4 * i < M)
+          e.extra[i] = __ldg(reinterpret_cast<const float4*>(p.rope_cs + (size_t)(r0 + 4 * i) * (p.head_dim >> 1) +
+                                                             pair));
+    }
+  } else if (p.epi == FSDIT_EPI_RESIDUAL) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (r0 + 4 * i < M) e.extra[i] = *reinterpret_cast<const float4*>(p.resid + (size_t)(r0 + 4 * i) * p.ldr + cl);
+  }
+}
+
+// The epilogue of the transposed block w (w[4i + j] = column cl + j of row
+// r0 + 4i): dequantization, bias, RoPE / GELU, then the residual add and the
+// store, or the unpatchify store.
+__device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col, int M, int lane, float* w,
+                                           const EpiTPre& e) {
+  const int cl = col + 4 * (lane & 7);
+  const int r0 = row0 + (lane >> 3);
+  if (p.col_scale != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[4 * i] *= e.rscale[i] * e.cscale.x;
+      w[4 * i + 1] *= e.rscale[i] * e.cscale.y;
+      w[4 * i + 2] *= e.rscale[i] * e.cscale.z;
+      w[4 * i + 3] *= e.rscale[i] * e.cscale.w;
+    }
+  }
+  {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&e.bias);
+    const float2 b01 = __bfloat1622float2(h[0]), b23 = __bfloat1622float2(h[1]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[4 * i] += b01.x;
+      w[4 * i + 1] += b01.y;
+      w[4 * i + 2] += b23.x;
+      w[4 * i + 3] += b23.y;
+    }
+  }
+  if (p.epi == FSDIT_EPI_QKV_ROPE) {
+    if (col < p.rope_cols && p.rope_cs == nullptr) {
+      // angles from the positions (rope_pair's arithmetic): the lane's two
+      // pairs keep their axis and frequency across its eight rows
+      int axis[2];
+      float inv_freq[2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int d = (cl + 2 * m) & (p.head_dim - 1);
+        int off, da;
+        if (d < p.s0) { axis[m] = 0; off = 0; da = p.s0; }
+        else if (d < p.s0 + p.s1) { axis[m] = 1; off = p.s0; da = p.s1; }
+        else { axis[m] = 2; off = p.s0 + p.s1; da = p.head_dim - p.s0 - p.s1; }
+        const float jj = (float)((d - off) >> 1);
+        inv_freq[m] = exp2f(-(2.0f * jj / (float)da) * p.log2_theta);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (r0 + 4 * i >= M) continue;
+        const int32_t* pos3 = p.pos + (size_t)(r0 + 4 * i) * 3;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const float ang = (float)__ldg(pos3 + axis[m]) * inv_freq[m];
+          float sn, cs;
+          sincosf(ang, &sn, &cs);
+          const float a = w[4 * i + 2 * m], b = w[4 * i + 2 * m + 1];
+          w[4 * i + 2 * m] = a * cs - b * sn;
+          w[4 * i + 2 * m + 1] = a * sn + b * cs;
+        }
+      }
+    } else if (col < p.rope_cols) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 t = e.extra[i];  // (cos, sin) of the lane's two pairs
+        float a = w[4 * i], b = w[4 * i + 1];
+        w[4 * i] = a * t.x - b * t.y;
+        w[4 * i + 1] = a * t.y + b * t.x;
+        a = w[4 * i + 2];
+        b = w[4 * i + 3];
+        w[4 * i + 2] = a * t.z - b * t.w;
+        w[4 * i + 3] = a * t.w + b * t.z;
+      }
+    }
+  } else if (p.epi == FSDIT_EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = gelu_tanh_bf16out(w[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = r0 + 4 * i;
+    if (row >= M) continue;
+    const float* x = w + 4 * i;
+    if (p.epi == EPI_UNPATCH) {
+      const long long off = unpatch_offset(p, row, cl);  // up_ps % 4 == 0: 4 adjacent pixels
+      if (off < 0) continue;
+      if (p.up_rgb8)
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.out) + off) =
+            rgb8_code(x[0]) | (rgb8_code(x[1]) << 8) | (rgb8_code(x[2]) << 16) | (rgb8_code(x[3]) << 24);
+      else
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + off) = make_float4(x[0], x[1], x[2], x[3]);
+    } else if (p.epi == FSDIT_EPI_RESIDUAL) {
+      const float4 r = e.extra[i];
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) =
+          make_float4(r.x + x[0], r.y + x[1], r.z + x[2], r.w + x[3]);
+    } else if (p.epi == FSDIT_EPI_BIAS_F32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) =
+          make_float4(x[0], x[1], x[2], x[3]);
+    } else {
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(x[2], x[3]);
+      *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(p.out) + (size_t)row * p.ldo + cl) =
+          make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+    }
+  }
+}
+
 }  // namespace fsdit
 
 // Host-side internal API shared by the .cu files.

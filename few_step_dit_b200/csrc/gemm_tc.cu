@@ -253,7 +253,12 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 // barrier ids: full[s] = s (rank 0's counts both CTAs' copies), empty[s] = S+s,
 // tfull[b] = 2S+b, tempty[b] = 2S+2+b (rank 0 only), drain = 2S+4
 constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
+// after the ring: barriers, TMEM address and abort flag, then each epilogue
+// warp's 4 KB block for warp_transpose32
+constexpr int EPI_OFF = STAGES * STAGE_BYTES + 1024;
+constexpr int SMEM_BYTES = EPI_OFF + EPI_WARPS * 4096 + 1024;
+static_assert(NUM_BARS * 8 + 16 <= 1024, "barrier block");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 constexpr int GROUP_N = 8;
 constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, 0);
 constexpr uint32_t IDESC_FP8 = ptx::idesc_e4m3(BM, BN);
@@ -467,6 +472,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // this warp's region of a tile: its rank's rows of lane quarter q, its
     // column half (the unit of the split-tail bookkeeping)
     const int region = ((int)rank * 4 + q) * 2 + (c0 != 0 ? 1 : 0);
+    float4* epi_buf = reinterpret_cast<float4*>(base_ptr + EPI_OFF) + (warp - 2) * 256;
     int it = 0;
     for (int u = cid; u < args.n_units; u += ncl, ++it) {
       int tile, kb0, kb1, sp, slot;
@@ -488,20 +494,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                             rank == 0 ? TEMPTY(buf) : tempty0 + 8u * (uint32_t)buf, rank == 0);
         continue;
       }
+      const int row0 = row - lane;  // first row of this warp's 32 x 32 blocks
 #pragma unroll 1
       for (int c = c0; c < c0 + BN / 64; ++c) {
         const int col = nb * BN + c * 32;
-        const bool full = row_ok && col + 32 <= args.N;
-        Epi32Pre pre;
-        if (full) epi32_prefetch(args.ep, row, col, pre);
         float v[32];
-        tmem_ld32(t_row + (uint32_t)(c * 32), v);
-        if (full) {
-          epi32_apply(args.ep, row, col, v, pre);
-        } else if (row_ok && col < args.N) {  // ragged last chunk (N % 32 != 0, N even)
+        if (col + 32 <= args.N) {  // warp-uniform: the block's columns are all inside
+          EpiTPre pre;
+          epiT_prefetch(args.ep, row0, col, args.M, lane, pre);
+          tmem_ld32(t_row + (uint32_t)(c * 32), v);
+          float w[32];
+          warp_transpose32(epi_buf, v, w, lane);
+          epiT_apply(args.ep, row0, col, args.M, lane, w, pre);
+        } else {
+          tmem_ld32(t_row + (uint32_t)(c * 32), v);
+          if (row_ok && col < args.N) {  // ragged last chunk (N % 32 != 0, N even)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
+            for (int i = 0; i < 32; i += 2)
+              if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
+          }
         }
       }
       tc_fence_before();
