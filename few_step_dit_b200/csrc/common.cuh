@@ -474,20 +474,48 @@ __device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col
 #pragma unroll
     for (int i = 0; i < 32; ++i) w[i] = gelu_tanh_bf16out(w[i]);
   }
+  if (p.epi == EPI_UNPATCH) {
+    // unpatch_offset's mapping with its divisions done once: the lane's
+    // columns fix (channel, dt, dy, dx) and its rows are the cells r0 + 4i,
+    // stepped four cells at a time through (t, h, w)
+    const int ps = p.up_ps, pt = p.up_pt;
+    const int dx = cl % ps, c1 = cl / ps;
+    const int dy = c1 % ps, c2 = c1 / ps;
+    const int dt = c2 % pt, ch = c2 / pt;
+    int cw = r0 % p.up_w, ct = r0 / p.up_w;
+    int chh = ct % p.up_h;
+    ct /= p.up_h;
+    const long long hp = (long long)p.up_h * ps, wp = (long long)p.up_w * ps;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int f = ct * pt + dt - (pt - 1);
+      if (r0 + 4 * i < M && f >= 0) {  // up_ps % 4 == 0: 4 adjacent pixels of one pixel row
+        const float* x = w + 4 * i;
+        const long long off =
+            (((long long)f * p.up_c + ch) * hp + (long long)chh * ps + dy) * wp + (long long)cw * ps + dx;
+        if (p.up_rgb8)
+          *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.out) + off) =
+              rgb8_code(x[0]) | (rgb8_code(x[1]) << 8) | (rgb8_code(x[2]) << 16) | (rgb8_code(x[3]) << 24);
+        else
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + off) = make_float4(x[0], x[1], x[2], x[3]);
+      }
+      cw += 4;
+      while (cw >= p.up_w) {  // at most 4 / up_w + 1 steps
+        cw -= p.up_w;
+        if (++chh == p.up_h) {
+          chh = 0;
+          ++ct;
+        }
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int row = r0 + 4 * i;
     if (row >= M) continue;
     const float* x = w + 4 * i;
-    if (p.epi == EPI_UNPATCH) {
-      const long long off = unpatch_offset(p, row, cl);  // up_ps % 4 == 0: 4 adjacent pixels
-      if (off < 0) continue;
-      if (p.up_rgb8)
-        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.out) + off) =
-            rgb8_code(x[0]) | (rgb8_code(x[1]) << 8) | (rgb8_code(x[2]) << 16) | (rgb8_code(x[3]) << 24);
-      else
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + off) = make_float4(x[0], x[1], x[2], x[3]);
-    } else if (p.epi == FSDIT_EPI_RESIDUAL) {
+    if (p.epi == FSDIT_EPI_RESIDUAL) {
       const float4 r = e.extra[i];
       *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) =
           make_float4(r.x + x[0], r.y + x[1], r.z + x[2], r.w + x[3]);
