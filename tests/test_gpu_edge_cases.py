@@ -54,6 +54,29 @@ def test_block_degenerate_sequences(grid, n_text, n_audio, compress):
     assert O.rel_l2(out.double().cpu().numpy() - xn, ref - xn) < 1e-5
 
 
+@pytest.mark.parametrize("dtype,bound", [("f32", 1e-5), ("bf16", 1e-2)])
+@pytest.mark.parametrize("split", [(34, 46, 48), (30, 50, 48)])
+def test_block_rope_split_with_odd_pair_counts(split, dtype, bound):
+    # chunk widths of 17 / 23 and 15 / 25 pairs: the RoPE table, the QKV
+    # epilogue and the oracle all take the axis of each pair from the split
+    w = _tiny(rope_split=split, dtype=dtype)
+    layers, _ = S.make_weights(w, n_layers=1)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    seq = api.Sequence.from_workload(w, tags, DEV, compress=True)
+    bw = api.BlockWeights({k: v.to(DEV) for k, v in layers[0].items()})
+    x = inp["x"].float()
+    out = api.block_forward(api.dims_of(w), bw, seq, x.to(DEV), compress=True)
+    torch.cuda.synchronize()
+    xn = x.double().numpy()
+    k, n = O.keep_map(*w.grid)
+    ref = O.dit_block_compressed(xn, S.to_numpy64(layers[0]), tags["pos"], w.heads, w.head_dim, k, n, w.n_video,
+                                 rope_split=split)
+    got = out.double().cpu().numpy()
+    assert O.rel_l2(got, ref) < bound
+    assert O.rel_l2(got - xn, ref - xn) < bound
+
+
 def test_one_token_grid_compression_keeps_everything():
     # a 1 x 1 x 1 grid keeps its only token: compressed block == plain block bit for bit
     w = _tiny(grid=(1, 1, 1))

@@ -175,6 +175,32 @@ def test_linear(dtype, M, N, K, epi):
         assert err < bound, err
 
 
+@pytest.mark.parametrize("split", [(34, 46, 48), (30, 50, 48), (32, 48, 48)])
+def test_linear_rope_chunks_with_odd_pair_boundaries(split):
+    # rope_split widths whose pair counts are odd put an axis boundary between
+    # the two pairs one lane rotates in the coalesced epilogue
+    g = _rng(12)
+    M, A, K = 300, 256, 256
+    dims = api.make_dims(A, A // 128, 512, torch.bfloat16, rope_split=split)
+    a = torch.randn(M, K, generator=g).bfloat16()
+    w = (0.05 * torch.randn(3 * A, K, generator=g)).bfloat16()
+    b = (0.05 * torch.randn(3 * A, generator=g)).bfloat16()
+    pos = torch.randint(0, 40, (M, 3), generator=g, dtype=torch.int32)
+    out = api.linear(dims, a.to(DEV), w.to(DEV), b.to(DEV), L.EPI_QKV_ROPE, pos=pos.to(DEV))
+    torch.cuda.synchronize()
+    y = O.linear(a.double().numpy(), w.double().numpy(), b.double().numpy())
+    q = O.apply_rope(y[:, :A].reshape(M, A // 128, 128), pos.numpy(), split).reshape(M, A)
+    k = O.apply_rope(y[:, A:2 * A].reshape(M, A // 128, 128), pos.numpy(), split).reshape(M, A)
+    ref = np.concatenate([q, k, y[:, 2 * A:]], axis=1)
+    assert O.rel_l2(_np(out), ref) < 5e-3
+    # the same split with the default one differs: the split reached the kernel
+    if split != (32, 48, 48):
+        ref0 = np.concatenate([O.apply_rope(y[:, :A].reshape(M, A // 128, 128), pos.numpy()).reshape(M, A),
+                               O.apply_rope(y[:, A:2 * A].reshape(M, A // 128, 128), pos.numpy()).reshape(M, A),
+                               y[:, 2 * A:]], axis=1)
+        assert O.rel_l2(_np(out), ref0) > 1e-2
+
+
 # ---------------------------------------------------------------- attention
 
 
