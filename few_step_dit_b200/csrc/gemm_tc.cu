@@ -209,7 +209,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 // commits release the stage in both CTAs.  Accumulator rows 0..127 of a tile
 // sit in rank 0's TMEM, 128..255 in rank 1's; each CTA's epilogue stores its
 // own rows and releases the accumulator buffer on rank 0's barrier (one arrive
-// per warp).  SPLIT = true instantiates the opt-in tail cut's second launch
+// per warp).  An epilogue warp takes 32 x 32 blocks out of TMEM one row per
+// lane and passes each through 4 KB of its own shared memory
+// (warp_transpose32), so that every global access of the epilogue then covers
+// four rows per instruction.  SPLIT = true instantiates the opt-in tail cut's second launch
 // (units of K-slices of the last wave's tiles, see split_unit_epilogue).
 namespace gemm2 {
 
