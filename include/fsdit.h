@@ -472,7 +472,10 @@ FSDIT_API fsdit_status fsdit_history_copy_frame(const fsdit_history_store* s, in
  * video modality, time id 0, not updated, pos left untouched (the gather
  * writes it).  Text rows: time id 0, pos (0,0,0).  Audio rows: time id 2,
  * updated, pos (floor(j T / n_audio) + base, 0, 0).  Host arrays of n =
- * T*H*W + n_hist + n_text + n_audio entries (pos: 3n). */
+ * T*H*W + n_hist + n_text + n_audio entries (pos: 3n).  Errors: FSDIT_E_NULL;
+ * FSDIT_E_SHAPE for a non-positive grid size, negative counts or base, or
+ * has_boundary with T < 2 (a chunk with a boundary frame has at least one new
+ * frame). */
 FSDIT_API fsdit_status fsdit_chunk_tags(int T, int H, int W, int base, int has_boundary, int n_hist, int n_text,
                                         int n_audio, uint8_t* modality, uint8_t* time_id, uint8_t* out_mask,
                                         int32_t* pos);
