@@ -184,9 +184,27 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int rows, int
 // precomputed text projection row.  Without tags (modality == nullptr: the
 // decoder's latent cells) x[r] = src(r).  A block owns EMB_RB rows of one segment
 // and EMB_CB consecutive columns: each thread keeps its column's weight row
-// in registers; the rows' latents, modality and timestep embeddings of the
-// block's columns are staged in shared memory; stores are coalesced.
+// in registers (each weight twice, as an f32x2 pair); the rows' latents are
+// staged channel-major in shared memory, so one 16-byte read gives a channel
+// of four rows and two packed FMAs advance four rows' sums (the same fma
+// sequence per output as a scalar loop over k); modality and timestep
+// embeddings of the block's columns are staged too; stores are coalesced.
 constexpr int EMB_RB = 128, EMB_CB = 256, EMB_MAXT = 8;
+
+typedef unsigned long long emb_f2;
+__device__ __forceinline__ emb_f2 emb_pair(float a, float b) {
+  emb_f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void emb_split(emb_f2 v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ emb_f2 emb_fma2(emb_f2 a, emb_f2 b, emb_f2 c) {
+  emb_f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 
 template <typename TW, int KMAX>
 __global__ void __launch_bounds__(256) embed_kernel(
@@ -195,7 +213,7 @@ __global__ void __launch_bounds__(256) embed_kernel(
     const float* __restrict__ text_proj, const TW* __restrict__ mod_emb, const float* __restrict__ temb,
     const uint8_t* __restrict__ modality, const uint8_t* __restrict__ time_id, int n_times,
     int expect_a, int expect_b) {
-  __shared__ float s_lat[EMB_RB][KMAX];
+  __shared__ __align__(16) float s_latT[KMAX][EMB_RB];  // channel-major: rows j..j+3 of channel k are one float4
   __shared__ float s_mod[4][EMB_CB];
   __shared__ float s_temb[EMB_MAXT][EMB_CB];
   __shared__ int s_m[EMB_RB], s_t[EMB_RB];
@@ -221,8 +239,8 @@ __global__ void __launch_bounds__(256) embed_kernel(
   }
   if (kind == 1) {
     for (int i = threadIdx.x; i < EMB_RB * KMAX; i += blockDim.x) {
-      const int rr = i / KMAX, kk = i % KMAX;
-      s_lat[rr][kk] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
+      const int rr = i % EMB_RB, kk = i / EMB_RB;  // consecutive threads: consecutive rows (no bank conflict)
+      s_latT[kk][rr] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
     }
   }
   if (tagged) {
@@ -232,24 +250,39 @@ __global__ void __launch_bounds__(256) embed_kernel(
   }
   __syncthreads();
   if (!col_ok) return;
-  float wr[KMAX];
-  float bias = 0.f;
   if (kind == 1) {
+    emb_f2 wd[KMAX];
 #pragma unroll
-    for (int k = 0; k < KMAX; ++k) wr[k] = k < K ? ld_f32<TW>(w_in + (size_t)c * K + k) : 0.f;
-    bias = ld_f32<TW>(b_in + c);
-  }
-  for (int j = 0; j < nr; ++j) {
-    float acc;
-    if (kind == 1) {
-      acc = bias;
-#pragma unroll
-      for (int k = 0; k < KMAX; ++k) acc = fmaf(s_lat[j][k], wr[k], acc);
-    } else {
-      acc = text_proj[(size_t)(rb0 + j) * hidden + c];
+    for (int k = 0; k < KMAX; ++k) {
+      const float wv = k < K ? ld_f32<TW>(w_in + (size_t)c * K + k) : 0.f;
+      wd[k] = emb_pair(wv, wv);
     }
-    if (tagged) acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
-    x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
+    const float bias = ld_f32<TW>(b_in + c);
+    for (int j = 0; j < nr; j += 4) {  // rows past nr are zero in s_latT and not stored
+      emb_f2 a01 = emb_pair(bias, bias), a23 = emb_pair(bias, bias);
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        const float4 l4 = *reinterpret_cast<const float4*>(&s_latT[k][j]);
+        a01 = emb_fma2(emb_pair(l4.x, l4.y), wd[k], a01);
+        a23 = emb_fma2(emb_pair(l4.z, l4.w), wd[k], a23);
+      }
+      float v[4];
+      emb_split(a01, v[0], v[1]);
+      emb_split(a23, v[2], v[3]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (j + u >= nr) break;
+        float acc = v[u];
+        if (tagged) acc += s_mod[s_m[j + u]][threadIdx.x] + s_temb[s_t[j + u]][threadIdx.x];
+        x[(size_t)(row0 + rb0 + j + u) * hidden + c] = acc;
+      }
+    }
+  } else {
+    for (int j = 0; j < nr; ++j) {
+      float acc = text_proj[(size_t)(rb0 + j) * hidden + c];
+      if (tagged) acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
+      x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
+    }
   }
 }
 
@@ -412,7 +445,11 @@ static fsdit_status embed_t(float* x, int hidden, int row0, int rows, int kind, 
                (double)rows * hidden * 4.0 * (kind == 0 ? 2.0 : 1.0) + (double)rows * K * 4.0 +
                    (double)hidden * K * sizeof(TW),
                st);
-  if (K <= 32)
+  if (K <= 24)
+    embed_kernel<TW, 24><<<grid, EMB_CB, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
+                                                  (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
+                                                  time_id, n_times, ea, eb);
+  else if (K <= 32)
     embed_kernel<TW, 32><<<grid, EMB_CB, 0, st>>>(x, hidden, row0, rows, kind, lat, K, (const TW*)w_in,
                                                   (const TW*)b_in, text_proj, (const TW*)mod_emb, temb, modality,
                                                   time_id, n_times, ea, eb);
