@@ -5,8 +5,6 @@ after its limit, the host reads FSDIT_E_TIMEOUT from the device error word,
 and the context keeps working (a projection afterwards is correct and the
 word is clear again)."""
 
-import ctypes as C
-
 import pytest
 import torch
 

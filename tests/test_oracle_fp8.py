@@ -4,7 +4,6 @@ quantizer's invariants, an exactly representable GEMM, and the quantized
 block against the full-precision block.  CPU only."""
 
 import numpy as np
-import pytest
 import torch
 
 import oracle as O
