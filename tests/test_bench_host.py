@@ -1,9 +1,8 @@
 """Host-side logic of bench.py, on CPU: the algorithmic FLOP counts behind the
 roofline figures (against per-layer and per-pass totals worked out by hand),
-the source hash that
-invalidates the recorded GEMM DRAM traffic when the GEMM code changes (and
-only then), and the parsing of the clock samples taken during the timed
-region."""
+the source hash that invalidates the recorded GEMM DRAM traffic when the GEMM
+code changes (and only then), and the parsing of the clock samples taken
+during the timed region."""
 
 import json
 import os
