@@ -124,7 +124,10 @@ typedef struct {
  *   grid_t/h/w: the target video grid, rows [0, grid_t*grid_h*grid_w) in
  *     (t,h,w) row-major order (0,0,0 if there is none); control rows follow.
  *   keep_idx [n_keep], near_idx [grid rows]: keep-index map of that grid from
- *     fsdit_build_keep_map (NULL/0: no compression).
+ *     fsdit_build_keep_map (NULL/0: no compression).  The kernels index with
+ *     these device arrays as they are: the host checks n_keep against the
+ *     grid, but entries that do not come from fsdit_build_keep_map (indices
+ *     outside the grid) are undefined behaviour.
  *   pos_thw [n_tokens][3] int32, modality/time_id/out_mask [n_tokens] uint8. */
 typedef struct {
   int n_tokens, n_vrows, n_text, n_audio;
