@@ -143,11 +143,18 @@ typedef struct {
 
 /* ---------------------------------------------------------------- queries */
 
+/* Message of this thread's last failed call (static storage of the thread,
+ * overwritten by its next failure; never NULL). */
 FSDIT_API const char* fsdit_last_error(void);
+/* Library name, version and target architecture (static string). */
 FSDIT_API const char* fsdit_version(void);
 
-/* Synchronizes `stream`, returns FSDIT_E_TIMEOUT if any kernel since the last
- * reset gave up a bounded wait (and clears the word), else FSDIT_OK. */
+/* Synchronizes `stream` and reads the device error word, which kernels set
+ * instead of trapping.  Returns FSDIT_E_TIMEOUT if a kernel gave up a bounded
+ * wait since the word was last cleared, FSDIT_E_SHAPE if the embedding found
+ * row tags inconsistent with the sequence's segments (modality or time slot
+ * out of place), else FSDIT_OK; a non-zero word is cleared and described in
+ * fsdit_last_error(). */
 FSDIT_API fsdit_status fsdit_device_error(fsdit_stream_t stream);
 
 /* Failure-path check (no fault): launches one thread that waits, through the
