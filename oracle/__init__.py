@@ -30,14 +30,18 @@ and ``decoder.py`` (the lightweight decoder's forward; ``oracle.decoder``).
 Every floating-point step runs in float64.  Where the pages leave a step open
 the plainest reading is taken; each one is marked ``Reading:`` in the docstring.
 
-Parity status per function: everything in ``dit.py`` is pinned by the CPU
-tests in ``tests/test_oracle_pins.py`` and everything in ``long_video.py`` by
-``tests/test_oracle_long_video.py``, everything in ``fp8.py`` by
-``tests/test_oracle_fp8.py`` and everything in ``decoder.py`` by
-``tests/test_oracle_decoder.py``, except the conventions that are pure
-definitions (weight init, time-embedding MLP, bias placement); those are
-"parity unpinned" in the sense that no page fixes them, so the GPU path is
-compared against this oracle's definition of them.
+Parity status per function: every public function is called by a named pin
+(``tests/test_oracle_composition.py`` checks that none is missing).  The
+pieces of ``dit.py`` are pinned in ``tests/test_oracle_pins.py``; its
+composites (the timestep MLP, the output heads, the stack with the Flash
+schedule and the sampler with its two clocks) in
+``tests/test_oracle_composition.py``, by weights that reduce each one to a
+closed form; ``long_video.py`` in ``tests/test_oracle_long_video.py``,
+``fp8.py`` in ``tests/test_oracle_fp8.py`` and ``decoder.py`` in
+``tests/test_oracle_decoder.py``.  Three conventions are definitions that no
+page fixes (the weight init, the timestep MLP's layer sizes and activation,
+which projections carry biases): the pins check the wiring the oracle gives
+them, and the GPU path is compared against that definition.
 """
 
 from .dit import *  # noqa: F401,F403

@@ -11,14 +11,12 @@ below is a reading:
   mantissa bits, subnormals, no infinity, largest finite 448).  Rounding is to
   nearest with ties to even; magnitudes beyond 448 saturate to 448.
 * Scaling: one fp32 scale per row of the operand that is quantized -- per
-  token for activations, per output channel for weights: s = amax / 448 (1
-  for an all-zero row), q = E4M3(value * r) with r = 1 / s, the scale's
-  reciprocal rounded to fp32 once per row (one multiply per value instead of
-  a division).  The amax, the reciprocal, the product and the rounding
-  decision are taken in fp32 (the kernels' precision), so both sides produce
-  the same codes from the same fp32 inputs; next to the exact quotient a
-  code moves only where value * r and value / s straddle an E4M3 rounding
-  midpoint (about 2^-20 of the values), by one step.
+  token for activations, per output channel for weights: s = amax / 448
+  (rounded to fp32, as a stored scale is; 1 for an all-zero row) and
+  q = E4M3(value / s), the quotient of the fp32 value by the fp32 scale taken
+  in float64 and rounded once to E4M3.  (A kernel may multiply by a rounded
+  reciprocal of s instead of dividing; its codes then differ from these only
+  where the two quotients straddle an E4M3 rounding midpoint, by one step.)
 * Which projections: the four of every block (QKV, O, FFN up, FFN down); the
   input/output embeddings, the time MLP and the heads stay as they are.
 * GEMM: out = (sum_k q_a q_w) * s_a[row] * s_w[col] + bias, then the
@@ -64,12 +62,11 @@ def quantize_rows(a):
     """Per-row E4M3 quantization of a [R, K] operand given in fp32.
 
     Returns (q [R, K] float64 holding E4M3 values, s [R] float64 holding the
-    fp32 scales) with a ~= q * s[:, None]."""
+    fp32 scales) with a ~= q * s[:, None]: s = fp32(amax / 448), q = E4M3(a / s)."""
     a32 = np.asarray(a, dtype=F32)
     amax = np.max(np.abs(a32), axis=1) if a32.shape[1] else np.zeros(a32.shape[0], F32)
     s = np.where(amax > 0, amax / F32(E4M3_MAX), F32(1.0)).astype(F32)
-    r = (F32(1.0) / s).astype(F32)
-    q = e4m3((a32 * r[:, None]).astype(F32))
+    q = e4m3(a32.astype(F64) / s.astype(F64)[:, None])
     return q, s.astype(F64)
 
 

@@ -174,3 +174,33 @@ def test_rgb8_is_monotone_and_within_half_a_code_of_the_exact_map():
     assert (np.diff(q) >= 0).all()
     exact = np.clip(127.5 * (v.astype(np.float64) + 1), 0, 255)
     assert (np.abs(q - exact) <= 0.5 + 1e-4).all()
+
+
+def test_decoder_tokens_without_blocks_is_the_latent_projection():
+    # no blocks: the hidden state of every cell is W_in z + b_in, cells in
+    # (t, h, w) row-major order; a zero block leaves it unchanged
+    rng = np.random.default_rng(8)
+    io = _io(rng, 256, 5, 3, 1, 2)
+    z = rng.standard_normal((2 * 3 * 2, 5))
+    x = D.decoder_tokens(z, [], io, 2, 3, 2, 2, 128)
+    np.testing.assert_allclose(x, z @ io["w_in"].T + io["b_in"], rtol=1e-13, atol=1e-13)
+    zero = {"w_qkv": np.zeros((768, 256)), "b_qkv": np.zeros(768), "w_o": np.zeros((256, 256)),
+            "b_o": np.zeros(256), "w_1": np.zeros((64, 256)), "b_1": np.zeros(64), "w_2": np.zeros((256, 64)),
+            "b_2": np.zeros(256), "g_attn": np.ones(256), "g_ffn": np.ones(256)}
+    np.testing.assert_array_equal(D.decoder_tokens(z, [zero], io, 2, 3, 2, 2, 128), x)
+
+
+def test_pixel_head_on_one_hot_rows():
+    # a row c e_j normalizes (eps = 0) to sign(c) sqrt(H) g_j e_j, so the head
+    # returns sign(c) sqrt(H) g_j W_out[:, j] + b_out; a missing gain or the
+    # head applied before the norm fails
+    rng = np.random.default_rng(9)
+    H = 16
+    io = _io(rng, H, 4, 3, 1, 2)
+    j, c = np.array([0, 7, 15]), np.array([3.0, -0.2, 40.0])
+    x = np.zeros((3, H))
+    x[np.arange(3), j] = c
+    got = D.pixel_head(x, io, eps=0.0)
+    for r in range(3):
+        want = np.sign(c[r]) * np.sqrt(H) * io["g_out"][j[r]] * io["w_out"][:, j[r]] + io["b_out"]
+        np.testing.assert_allclose(got[r], want, rtol=1e-12, atol=1e-12)

@@ -67,18 +67,45 @@ def test_quantize_rows_invariants():
     np.testing.assert_array_equal(s.astype(np.float32).astype(np.float64), s)
 
 
-def test_quantize_rows_reciprocal_codes_are_the_exact_quotients_codes_but_at_midpoints():
-    # the codes come from value * fp32(1/s); against the E4M3 rounding of the
-    # exact quotient value / s (computed in float64) a code may differ only
-    # where the two straddle a rounding midpoint: rarely, and by one step
-    rng = np.random.default_rng(11)
-    a = (rng.standard_normal((200, 4096)) * rng.uniform(0.01, 50, (200, 1))).astype(np.float32)
+def _reciprocal_multiply_codes(a):
+    """The kernels' form of the quantizer, restated here (not in the oracle):
+    the row scale s = fp32(amax / 448) as in the definition, then every value
+    multiplied by r = fp32(1 / s) in fp32 and that product rounded to E4M3."""
+    a32 = np.asarray(a, dtype=np.float32)
+    amax = np.abs(a32).max(axis=1)
+    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    r = (np.float32(1.0) / s).astype(np.float32)
+    return Q.e4m3((a32 * r[:, None]).astype(np.float32)), s
+
+
+def test_quantize_rows_is_the_plain_quotient():
+    # the definition itself on values whose quotient is exact: a row whose
+    # amax is 448 has scale 1, and its codes are the E4M3 roundings of the
+    # values themselves
+    a = np.array([[448.0, 1.0, -3.3, 0.0137, 100.0, -448.0, 5e-4, 17.25]], dtype=np.float32)
     q, s = Q.quantize_rows(a)
-    exact = Q.e4m3(a.astype(np.float64) / s[:, None])
-    diff = q != exact
-    assert diff.mean() < 1e-4
-    step = np.maximum(np.abs(exact[diff]) * 2.0 ** -3, 2.0 ** -9)
-    assert (np.abs(q[diff] - exact[diff]) <= step * (1 + 1e-9)).all()
+    assert s[0] == 1.0
+    np.testing.assert_array_equal(q[0], Q.e4m3(a[0].astype(np.float64)))
+    # scale 2^k: dividing by a power of two is exact, codes shift by binades
+    q2, s2 = Q.quantize_rows(a * np.float32(8.0))
+    assert s2[0] == 8.0
+    np.testing.assert_array_equal(q2, q)
+
+
+def test_reciprocal_multiply_form_moves_at_most_one_step_on_at_most_2_pow_minus_16_of_values():
+    # A kernel that multiplies by fp32(1/s) instead of dividing may round a
+    # value to the neighbouring code where v*r and v/s straddle an E4M3
+    # midpoint.  Bound it: one step (1/8 of the value in a normal binade, the
+    # subnormal quantum 2^-9 below it), on at most 2^-16 of the values.
+    rng = np.random.default_rng(11)
+    a = (rng.standard_normal((400, 4096)) * rng.uniform(0.01, 50, (400, 1))).astype(np.float32)
+    q, s = Q.quantize_rows(a)
+    qk, sk = _reciprocal_multiply_codes(a)
+    np.testing.assert_array_equal(sk.astype(np.float64), s)
+    diff = qk != q
+    assert diff.sum() <= a.size * 2.0 ** -16, diff.sum()
+    step = np.maximum(np.abs(q[diff]) * 2.0 ** -3, 2.0 ** -9)
+    assert (np.abs(qk[diff] - q[diff]) <= step * (1 + 1e-9)).all()
 
 
 def test_linear_fp8_exact_on_representable_operands():
@@ -158,3 +185,19 @@ def test_fp8_block_row_restriction_equals_the_block():
     fullc = O.dit_block_compressed(x, w, pos_g, 2, 128, k, nn, n, block_fn=Q.dit_block_fp8)
     got = O.dit_block_compressed_rows(x, w, pos_g, 2, 128, k, nn, n, rows, rows_fn=Q.dit_block_fp8_rows)
     np.testing.assert_allclose(got, fullc[rows], rtol=1e-10, atol=1e-12)
+
+
+def test_quantize_block_weights_quantizes_each_projection_per_output_channel():
+    # the four projections, each row (output channel) with its own scale; a
+    # row whose largest magnitude is 448 keeps scale 1 and its values' codes
+    rng = np.random.default_rng(12)
+    w = {"w_qkv": rng.standard_normal((6, 4)), "w_o": rng.standard_normal((4, 2)),
+         "w_1": rng.standard_normal((3, 4)), "w_2": rng.standard_normal((4, 3)), "b_o": np.zeros(4)}
+    w["w_o"][1] = [448.0, -5.0]
+    wq = Q.quantize_block_weights(w)
+    assert sorted(wq) == ["w_1", "w_2", "w_o", "w_qkv"]
+    for k, (q, s) in wq.items():
+        assert q.shape == w[k].shape and s.shape == (w[k].shape[0],)
+        np.testing.assert_array_equal(s, np.abs(w[k]).max(axis=1).astype(np.float32) / np.float32(448.0))
+    assert wq["w_o"][1][1] == 1.0
+    np.testing.assert_array_equal(wq["w_o"][0][1], Q.e4m3(np.array([448.0, -5.0])))

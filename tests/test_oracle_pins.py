@@ -520,3 +520,26 @@ def test_embed_routes_rows_by_modality():
     np.testing.assert_allclose(x[5, :5], 2 * te[1] + base[:5])
     np.testing.assert_allclose(x[4, :4], 3 * al[0] + 100 + base[:4])
     np.testing.assert_allclose(x[4, 4:], 100 + base[4:])
+
+
+def test_axis_nearest_printed_axes():
+    # the 9 x 10 example: rows keep {0,2,4,6,8}, columns {0,2,4,6,8,9}; every
+    # dropped index takes the kept index just below it (ties -> lower)
+    assert O.axis_nearest(9) == [0, 0, 2, 2, 4, 4, 6, 6, 8]
+    assert O.axis_nearest(10) == [0, 0, 2, 2, 4, 4, 6, 6, 8, 9]
+    assert O.axis_nearest(1) == [0] and O.axis_nearest(2) == [0, 1]
+
+
+def test_rope_angles_per_axis_frequencies():
+    # position (1, 0, 0) turns only the t chunk (16 pairs) by theta^(-2j/32);
+    # (0, 1, 0) only the h chunk (24 pairs) by theta^(-2j/48); (0, 0, 2) the w
+    # chunk by 2 theta^(-2j/48)
+    ang = O.rope_angles(np.array([[1, 0, 0], [0, 1, 0], [0, 0, 2]]))
+    assert ang.shape == (3, 64)
+    jt, jh = np.arange(16), np.arange(24)
+    np.testing.assert_allclose(ang[0, :16], 10000.0 ** (-2 * jt / 32), rtol=1e-14)
+    np.testing.assert_array_equal(ang[0, 16:], 0)
+    np.testing.assert_array_equal(ang[1, :16], 0)
+    np.testing.assert_allclose(ang[1, 16:40], 10000.0 ** (-2 * jh / 48), rtol=1e-14)
+    np.testing.assert_array_equal(ang[1, 40:], 0)
+    np.testing.assert_allclose(ang[2, 40:], 2 * 10000.0 ** (-2 * jh / 48), rtol=1e-14)
