@@ -46,6 +46,8 @@ def metric_of(w):
 UNIT = "tokens/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's dense bf16 tensor-core figure for one B200 (context for the fractions)
+NOMINAL_BF16_TFLOPS = 2250.0
 GEMM_SOURCES = ["few_step_dit_b200/csrc/gemm_tc.cu", "few_step_dit_b200/csrc/common.cuh",
                 "few_step_dit_b200/csrc/tc_ptx.cuh"]
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "gemm_traffic_flash_backbone_6x34x60.json")
@@ -109,6 +111,17 @@ def gemm_traffic(workload):
     if d.get("workload") != workload or d.get("sources_sha256") != gemm_sources_sha256():
         return None
     return d.get("dram_bytes_per_launch")
+
+
+def peak_fracs(achieved, sustained, burst, nominal=None):
+    """A TFLOP/s figure as a fraction of each basis: the measured sustained
+    (power-capped, seconds-long) cuBLAS rate, the measured burst rate, and the
+    nominal dense peak."""
+    nominal = NOMINAL_BF16_TFLOPS if nominal is None else nominal
+    out = {"of_measured_sustained": achieved / sustained if sustained else None,
+           "of_measured_burst": achieved / burst if burst else None,
+           "of_nominal_dense": achieved / nominal if nominal else None}
+    return out
 
 
 # ---------------------------------------------------------------- clocks
@@ -212,10 +225,46 @@ def oracle_sample(w, reps=1):
     for c in w.compress:
         per_pass += t_s * block_flops(w, n_s if c else w.n_tokens) / f_s
     per_pass *= w.n_evals
-    desc = (f"one {'token-compressed ' if comp else ''}full-width block ({n_s} rows, hidden {w.hidden}) "
-            f"timed in fp64 numpy ({t_s:.2f} s); other layers scaled by FLOPs; pass = {w.n_evals} evals x "
+    desc = (f"projected by FLOPs from one {'token-compressed ' if comp else ''}full-width block ({n_s} rows, "
+            f"hidden {w.hidden}) timed in fp64 numpy ({t_s:.2f} s); pass = {w.n_evals} evals x "
             f"({n_comp} compressed + {len(w.compress) - n_comp} full layers)")
     return w.n_tokens * w.n_evals / per_pass, per_pass, desc, blas_threads()
+
+
+def oracle_tiny(reps=3):
+    """The oracle timed directly (no projection) on the tiny fp32 workload:
+    one compressed block, one plain block and one Euler step (video
+    0.2 -> 0.0769, audio 0.5 -> 0.25), median of `reps`."""
+    import numpy as np
+
+    import oracle as O
+
+    w = S.WORKLOADS["tiny_block_f32"]
+    g = torch.Generator().manual_seed(S.SEED_WEIGHTS)
+    wts = S.to_numpy64(S.make_block_weights(w, g))
+    tags = S.pack_tokens(w)
+    inp = S.make_inputs(w)
+    x = inp["x"].double().numpy()
+    k, near = O.keep_map(*w.grid)
+    vl = inp["video_lat"].double().numpy()
+    v = np.ones_like(vl)
+    mods = tags["modality"][:vl.shape[0]]
+    mask = tags["out_mask"][:vl.shape[0]]
+
+    def med(fn):
+        ts = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            fn()
+            ts.append(time.perf_counter() - t0)
+        return statistics.median(ts) * 1e3
+
+    comp = med(lambda: O.dit_block_compressed(x, wts, tags["pos"], w.heads, w.head_dim, k, near, w.n_video))
+    plain = med(lambda: O.dit_block(x, wts, tags["pos"], w.heads, w.head_dim))
+    eul = med(lambda: O.euler_step(vl, v, mods, mask, [0, 0.2, 0.5, 0], [0, 0.0769, 0.25, 0]))
+    return {"workload": "tiny_block_f32", "tokens": w.n_tokens, "compressed_block_ms": comp,
+            "block_ms": plain, "euler_step_ms": eul, "tokens_per_s_block": w.n_tokens / (plain / 1e3),
+            "cores": blas_threads(), "timed": "directly, median of %d" % reps}
 
 
 def blas_threads():
@@ -309,9 +358,10 @@ def run_fsdit(args, rank, world, local_rank):
     api.device_error()
     R.barrier(world, device)
 
-    # capture one pass in a CUDA graph; the library's event profiler is active
-    # during the capture, so its event pairs replay with every launch
-    L.profile_start(20000)
+    # Timed region: one pass captured in a CUDA graph with the library's
+    # launch profiler off, replayed K times.  The per-kernel breakdown comes
+    # from a second graph of the same pass captured with the profiler on (its
+    # event pairs replay with every launch), replayed once after the timing.
     graph, launch_mode = None, "eager"
     if not args.eager:
         try:
@@ -322,8 +372,6 @@ def run_fsdit(args, rank, world, local_rank):
         except Exception as e:  # noqa: BLE001
             launch_mode = f"eager (graph capture failed: {type(e).__name__})"
             torch.cuda.synchronize()
-            L.profile_stop()
-            L.profile_start(20000)
     run = graph.replay if graph is not None else step
     if graph is not None:
         run()  # one untimed replay
@@ -333,13 +381,31 @@ def run_fsdit(args, rank, world, local_rank):
     t_ms = timed(run, args.steps, stream)
     R.barrier(world, device)
     clk = clocks.stop()
-    prof = L.profile_stop()  # the last pass's launches (graph) / all passes (eager)
-    prof_steps = 1 if graph is not None else args.steps
     api.device_error()
     t_ms = R.max_over_ranks(t_ms, world, device)
     ms_per_step = t_ms / args.steps
     value = R.weak_scaling_value(w.n_tokens * w.n_evals, world, ms_per_step / 1000.0)
     del graph
+
+    # the instrumented pass: per-kernel times, FLOPs and bytes
+    L.profile_start(20000)
+    prof_graph = None
+    if launch_mode == "cuda_graph":
+        prof_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(prof_graph):
+            step()
+        prof_graph.replay()
+    else:
+        step()
+    torch.cuda.synchronize()
+    # the replay's own duration, next to the clean pass (the event pairs' cost)
+    prof_ms = None
+    if prof_graph is not None:
+        prof_ms = timed(prof_graph.replay, 1, stream)
+    prof = L.profile_stop()  # the last replay's launches
+    prof_steps = 1
+    del prof_graph
+    api.device_error()
 
     # end to end through the public API: pinned host inputs -> device, sample, result -> host
     pin = {k: v.pin_memory() for k, v in inp.items() if k in ("video_lat", "audio_lat", "text_emb")}
@@ -369,6 +435,7 @@ def run_fsdit(args, rank, world, local_rank):
         full_ms = R.max_over_ranks(timed(lambda: step(False), n_full, stream), world, device) / n_full
 
     peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     gemm = {k: v for k, v in prof.items() if k.startswith("gemm")}
     g_ms = sum(v["ms"] for v in gemm.values())
     g_fl = sum(v["flops"] for v in gemm.values())
@@ -400,6 +467,7 @@ def run_fsdit(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: the bf16 weights (22.7 GB for 42 layers) stream from HBM "
                          "every evaluation"},
         "tensor_peak_frac": (pass_flops(w) / (ms_per_step / 1e3) / 1e12) / peak,
+        "tensor_peak_fracs": peak_fracs(pass_flops(w) / (ms_per_step / 1e3) / 1e12, peak, burst),
         "roofline": {"bound": "tensor", "kernel": "tc_gemm_pair_kernel (all projections with M > 128)"
                      + (", E4M3 operands" if args.proj_fp8 else ""),
                      "achieved": achieved, "peak": gemm_peak, "unit": "TFLOP/s",
@@ -407,12 +475,16 @@ def run_fsdit(args, rank, world, local_rank):
                      "traffic": None if args.proj_fp8 else gemm_traffic(args.workload),
                      "peak_source": f"{peak_src} bf16_tflops_sustained" + (" x 2 (E4M3/bf16 nominal ratio)"
                                                                            if args.proj_fp8 else ""),
-                     "launches_per_step": g_n // prof_steps},
+                     "launches_per_step": g_n // prof_steps,
+                     "fracs": peak_fracs(achieved, gemm_peak, (2.0 if args.proj_fp8 else 1.0) * burst,
+                                         (2.0 if args.proj_fp8 else 1.0) * NOMINAL_BF16_TFLOPS)},
         "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": R.weak_scaling_value(w.n_tokens * w.n_evals, world, e_ms / 1000.0), "unit": UNIT,
                 "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
+    if prof_ms is not None:
+        line["profiled_ms_per_step"] = prof_ms
     if full_ms is not None:
         line["uncompressed_ms_per_step"] = full_ms
         line["compression_speedup"] = full_ms / ms_per_step
@@ -426,7 +498,7 @@ def run_fsdit(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.proj_fp8:
         v, _, desc, threads = oracle_sample(w)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "projected": True, "tiny": oracle_tiny()}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

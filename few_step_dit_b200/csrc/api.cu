@@ -96,15 +96,17 @@ fsdit_status cuda_check(cudaError_t e, const char* what) {
 }
 
 int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-      n = v;
-    if (n <= 0) n = 148;
-  });
-  return n;
+  static PerDevice<int> sms;
+  return sms.get(
+      [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+          return v;
+        (void)cudaGetLastError();
+        return 148;
+      },
+      148);
 }
 
 #define FS_TRY(expr)                        \
@@ -468,8 +470,10 @@ fsdit_status fsdit_device_error(fsdit_stream_t stream) {
   if (v != 0) {
     int z = 0;
     FS_TRY(cuda_check(cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)), "clear device error word"));
-    set_error("device error word 0x%x (%s%s)", v, (v & DEVERR_TIMEOUT) ? "bounded wait timed out " : "",
-              (v & DEVERR_TAGS) ? "row tags inconsistent with segments" : "");
+    set_error("device error word 0x%x (%s%s%s)", v, (v & DEVERR_TIMEOUT) ? "bounded wait timed out; " : "",
+              (v & DEVERR_TAGS) ? "row tags inconsistent with segments; " : "",
+              (v & DEVERR_KEEPMAP) ? "keep_idx / near_idx entry outside the grid or not a nearest-kept map; "
+                                   : "");
     return (v & DEVERR_TIMEOUT) ? FSDIT_E_TIMEOUT : FSDIT_E_SHAPE;
   }
   return FSDIT_OK;

@@ -339,11 +339,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int attn_w, cudaStream_t st) {
   using namespace attn;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
+  static PerDevice<cudaError_t> attr;
+  const cudaError_t attr_err = attr.get(
+      [] { return cudaFuncSetAttribute(tc_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES); },
+      cudaErrorInvalidDevice);
   if (attr_err != cudaSuccess) return cuda_check(attr_err, "cudaFuncSetAttribute(tc_attention_kernel)");
   CUtensorMap tm;
   fsdit_status s = make_tmap_bf16(&tm, qkv, (uint64_t)n, (uint64_t)3 * attn_w, (uint64_t)3 * attn_w, BQ, 64);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/fsdit.h"
 
 namespace fsdit {
@@ -15,9 +17,36 @@ typedef __nv_bfloat16 bf16;
 // reads it through fsdit_device_error().
 __device__ int g_device_error = 0;  // one translation unit (libfsdit.cu) includes every source
 
-enum { DEVERR_TIMEOUT = 1, DEVERR_TAGS = 2 };
+enum { DEVERR_TIMEOUT = 1, DEVERR_TAGS = 2, DEVERR_KEEPMAP = 4 };
 
 __device__ __forceinline__ void raise_device_error(int code) { atomicOr(&g_device_error, code); }
+
+// Host-side values that belong to one device's context (kernel attributes,
+// occupancy, SM count) are computed once per device, on first use with that
+// device current, so a process may drive several GPUs.
+constexpr int MAX_DEVICES = 64;
+template <typename T>
+struct PerDevice {
+  std::mutex mu;
+  bool done[MAX_DEVICES] = {};
+  T val[MAX_DEVICES] = {};
+  // `init` runs with the device current; `on_error` is returned when the
+  // current device cannot be read or lies beyond MAX_DEVICES.
+  template <typename F>
+  T get(F init, T on_error) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+      (void)cudaGetLastError();
+      return on_error;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+      val[dev] = init();
+      done[dev] = true;
+    }
+    return val[dev];
+  }
+};
 
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
 template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }

@@ -31,7 +31,9 @@ __global__ void keep_map_kernel(int T, int H, int W, int32_t* __restrict__ keep_
 
 // ---------------------------------------------------------------- gather
 
-// One block per output row (grid-stride over rows); float4 copies.
+// One block per output row (grid-stride over rows); float4 copies.  A keep
+// index outside [0, n_grid) is not followed: the row is left as it is and the
+// device error word records DEVERR_KEEPMAP.
 __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* __restrict__ pos,
                                    float* __restrict__ xc, int32_t* __restrict__ posc,
                                    const int32_t* __restrict__ keep_idx, int n_keep, int n_grid,
@@ -39,6 +41,10 @@ __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* _
   const int h4 = hidden >> 2;
   for (int r = blockIdx.x; r < n_out; r += gridDim.x) {
     const int src = r < n_keep ? keep_idx[r] : n_grid + (r - n_keep);
+    if (r < n_keep && (src < 0 || src >= n_grid)) {
+      if (threadIdx.x == 0) raise_device_error(DEVERR_KEEPMAP);
+      continue;
+    }
     const float4* s = reinterpret_cast<const float4*>(x + (size_t)src * hidden);
     float4* d = reinterpret_cast<float4*>(xc + (size_t)r * hidden);
     for (int i = threadIdx.x; i < h4; i += blockDim.x) d[i] = __ldg(s + i);
@@ -54,9 +60,33 @@ __global__ void gather_rows_kernel(const float* __restrict__ x, const int32_t* _
 // reads y_c[b] and x[src] once: out[src] = y_c[b], out[p] = x[p] + (y_c[b] -
 // x[src]) for the others.  No two blocks touch the same row, so out may equal
 // x.  Blocks b >= n_keep copy the non-grid rows (text, audio, control).
+//
+// The maps are checked as they are used, so a map that does not come from
+// fsdit_build_keep_map is never followed out of bounds and never leaves a row
+// silently unwritten: a block skips its token when keep_idx[b] is outside the
+// grid or near_idx[keep_idx[b]] != b (a kept row must map to itself; this
+// also makes keep_idx injective), and every thread checks grid rows p in a
+// grid-stride loop: near_idx[p] must name a kept token c whose row lies in
+// p's frame, at most one row above and one column left of p.  Together these
+// are exactly the conditions under which every grid row is written once.  A
+// failed check sets DEVERR_KEEPMAP in the device error word.
+__device__ __forceinline__ bool near_entry_ok(const int32_t* keep_idx, const int32_t* near_idx, int p, int n_keep,
+                                              int grid_h, int grid_w, int n_grid) {
+  const int c = near_idx[p];
+  if (c < 0 || c >= n_keep) return false;
+  const int s = keep_idx[c];
+  if (s < 0 || s >= n_grid) return false;
+  const int hw = grid_h * grid_w;
+  if (s / hw != p / hw) return false;
+  const int dh = (p % hw) / grid_w - (s % hw) / grid_w, dw = p % grid_w - s % grid_w;
+  return dh >= 0 && dh <= 1 && dw >= 0 && dw <= 1;
+}
+
 __global__ void broadcast_kernel(const float* x, const float* __restrict__ yc, float* out,
                                  const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ near_idx,
                                  int n_keep, int grid_h, int grid_w, int n_grid, int n_rows, int hidden) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n_grid; p += gridDim.x * blockDim.x)
+    if (!near_entry_ok(keep_idx, near_idx, p, n_keep, grid_h, grid_w, n_grid)) raise_device_error(DEVERR_KEEPMAP);
   const int h4 = hidden >> 2;
   const int n_blocks = n_keep + (n_rows - n_grid);
   for (int b = blockIdx.x; b < n_blocks; b += gridDim.x) {
@@ -67,6 +97,10 @@ __global__ void broadcast_kernel(const float* x, const float* __restrict__ yc, f
       continue;
     }
     const int src = keep_idx[b];
+    if (src < 0 || src >= n_grid || near_idx[src] != b) {
+      if (threadIdx.x == 0) raise_device_error(DEVERR_KEEPMAP);
+      continue;
+    }
     const int w = src % grid_w, h = (src / grid_w) % grid_h;
     int child[3];
     int nc = 0;

@@ -596,15 +596,15 @@ fsdit_status make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t rows, uint6
 }
 
 static int pair_clusters_resident() {
-  static std::once_flag once;
-  static int n = 0;
-  std::call_once(once, [] {
+  static PerDevice<int> resident;
+  return resident.get([] {
+    int n = 0;
     for (auto fn : {gemm2::tc_gemm_pair_kernel<false, false>, gemm2::tc_gemm_pair_kernel<true, false>,
                     gemm2::tc_gemm_pair_kernel<false, true>, gemm2::tc_gemm_pair_kernel<true, true>}) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
         (void)cudaGetLastError();
-        return;
+        return 0;
       }
     }
     cudaLaunchConfig_t cfg = {};
@@ -621,8 +621,8 @@ static int pair_clusters_resident() {
     int c = 0;
     if (cudaOccupancyMaxActiveClusters(&c, gemm2::tc_gemm_pair_kernel<false, false>, &cfg) == cudaSuccess) n = c;
     (void)cudaGetLastError();
-  });
-  return n;
+    return n;
+  }, 0);
 }
 
 static fsdit_status launch_linear_pair(const void* a, const void* w, const EpiParams& ep, int M, int N, int K,
@@ -725,11 +725,10 @@ fsdit_status launch_linear_tc(const void* a, const void* w, const EpiParams& ep,
     if (clusters > 0) return launch_linear_pair(a, w, ep, M, N, K, clusters, false, st);
   }
   using namespace gemm;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
+  static PerDevice<cudaError_t> attr;
+  const cudaError_t attr_err = attr.get(
+      [] { return cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES); },
+      cudaErrorInvalidDevice);
   if (attr_err != cudaSuccess) return cuda_check(attr_err, "cudaFuncSetAttribute(tc_gemm_kernel)");
   CUtensorMap tmA, tmB;
   fsdit_status s = make_tmap_bf16(&tmA, a, (uint64_t)M, (uint64_t)K, (uint64_t)K, BM, BK);

@@ -48,23 +48,30 @@ extern "C" fsdit_status dit_block_forward_noalloc(const fsdit_dims* dims, const 
                                                   const fsdit_tokens* tok, const float* x_in, float* x_out,
                                                   fsdit_stream_t stream) {
   using namespace fsdit;
-  if (dims == nullptr || tok == nullptr) {
-    set_error("noalloc: dims and tokens are required");
-    return FSDIT_E_NULL;
-  }
-  const size_t need = fsdit_block_workspace_size(dims, tok->n_tokens, tok->keep_idx != nullptr ? tok->n_keep : 0);
-  if (need == 0) {
-    set_error("noalloc: invalid dims or token count");
-    return FSDIT_E_SHAPE;
-  }
-  if (need > NOALLOC_SCRATCH_BYTES) {
+  FS_TRY(check_dims(dims));
+  FS_TRY(check_block_weights(dims, w));
+  FS_TRY(check_tokens(tok, false));
+  // the scratch this block takes: the same carve as dit_block_forward, with
+  // the block's real compressed row count
+  const bool comp = tok->keep_idx != nullptr;
+  Carve c{nullptr, 0};
+  carve_block(c, dims, tok->n_tokens, comp ? n_compressed(tok) : tok->n_tokens, comp);
+  if (c.off > NOALLOC_SCRATCH_BYTES) {
     set_error("noalloc: this block needs %zu bytes of scratch, more than the %zu-byte static array; "
               "use dit_block_forward with a caller-provided workspace",
-              need, NOALLOC_SCRATCH_BYTES);
+              c.off, NOALLOC_SCRATCH_BYTES);
     return FSDIT_E_WORKSPACE;
   }
+  // the array is looked up for the current device, so the stream must be one of its streams
+  int cur = 0, sdev = 0;
+  FS_TRY(cuda_check(cudaGetDevice(&cur), "cudaGetDevice"));
+  FS_TRY(cuda_check(cudaStreamGetDevice((cudaStream_t)stream, &sdev), "cudaStreamGetDevice"));
+  if (sdev != cur) {
+    set_error("noalloc: the stream belongs to device %d but device %d is current; make the stream's device current",
+              sdev, cur);
+    return FSDIT_E_CUDA;
+  }
   void* scratch = nullptr;
-  fsdit_status s = noalloc_scratch_address(&scratch);
-  if (s != FSDIT_OK) return s;
+  FS_TRY(noalloc_scratch_address(&scratch));
   return dit_block_forward(dims, w, tok, x_in, x_out, scratch, NOALLOC_SCRATCH_BYTES, stream);
 }

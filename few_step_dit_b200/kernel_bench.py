@@ -6,6 +6,8 @@ Examples:
   python -m few_step_dit_b200.kernel_bench block --workload flash_block_6x34x60
   python -m few_step_dit_b200.kernel_bench decoder [--grid 6x34x60] [--fp8]
   python -m few_step_dit_b200.kernel_bench generate   # 3-eval Flash pass + decoder
+  python -m few_step_dit_b200.kernel_bench sweep      # compression sweep, 3 grids
+  python -m few_step_dit_b200.kernel_bench layer --M 3668   # one layer's four projections
 Inputs are seeded Gaussians; each case prints one JSON line.
 """
 
@@ -277,9 +279,97 @@ def case_generate(a):
             "frames_per_s": wd.n_frames / ms * 1e3}
 
 
+SWEEP_GRIDS = ("6x17x30", "6x34x60", "12x34x60")
+
+
+def case_sweep(a):
+    """The compression sweep: one full-width Flash block (hidden 5376, 56 x
+    128 heads, FFN 14336, bf16, 256 text + 64 audio rows) at each video grid,
+    compressed (per-block form: gather, block on the kept rows, nearest-kept
+    broadcast) and uncompressed.  Per grid: kept count, ms per block from a
+    CUDA graph, and from one profiled run of each form the GEMM and attention
+    TFLOP/s and the gather / broadcast GB/s.  Prints one JSON line per grid."""
+    grids = a.grids.split(",") if a.grids else SWEEP_GRIDS
+    out = []
+    w0 = S.WORKLOADS["flash_block_6x34x60"]
+    layers, _ = S.make_weights(w0, device="cuda", n_layers=1)
+    bw = api.BlockWeights(layers[0])
+    dims = api.dims_of(w0)
+    for gname in grids:
+        w = S.scaled(w0, grid=tuple(int(v) for v in gname.split("x")))
+        seq = api.Sequence.from_workload(w, S.pack_tokens(w), "cuda", compress=True)
+        g = torch.Generator(device="cuda").manual_seed(4)
+        x = torch.randn(w.n_tokens, w.hidden, generator=g, device="cuda")
+        y = torch.empty_like(x)
+        res = {"case": "sweep", "workload": f"flash_block_{gname}", "tokens": w.n_tokens,
+               "video_tokens": w.n_video, "kept_video_tokens": seq.n_keep, "compressed_tokens": seq.n_compressed}
+        for comp in (False, True):
+            tag = "compressed" if comp else "full"
+            step = lambda: api.block_forward(dims, bw, seq, x, y, compress=comp)  # noqa: E731
+            res[f"ms_{tag}"] = _graph_ms(step, a)
+            prof = _profile(step)
+            gm = {k: v for k, v in prof.items() if k.startswith("gemm")}
+            g_ms = sum(v["ms"] for v in gm.values())
+            g_fl = sum(v["tflops"] * v["ms"] * 1e9 for v in gm.values() if v["tflops"])
+            res[f"gemm_tflops_{tag}"] = round(g_fl / g_ms / 1e9, 1) if g_ms else None
+            if "attention" in prof:
+                res[f"attention_tflops_{tag}"] = prof["attention"]["tflops"]
+                res[f"attention_ms_{tag}"] = prof["attention"]["ms"]
+            res[f"gemm_ms_{tag}"] = round(g_ms, 3)
+            for k in ("gather", "broadcast", "rmsnorm_cast"):
+                if k in prof:
+                    res[f"{k}_gbs_{tag}"] = prof[k]["gbs"]
+                    res[f"{k}_ms_{tag}"] = prof[k]["ms"]
+        A, H, F = w.attn_dim, w.hidden, w.ffn
+
+        def fl(n):
+            return 2.0 * n * (4 * A * H + 2 * H * F) + 4.0 * n * n * A
+
+        res["tflop_full"] = fl(w.n_tokens) / 1e12
+        res["tflop_compressed"] = fl(seq.n_compressed) / 1e12
+        res["tflops_full"] = res["tflop_full"] / res["ms_full"] * 1e3
+        res["tflops_compressed"] = res["tflop_compressed"] / res["ms_compressed"] * 1e3
+        res["speedup"] = res["ms_full"] / res["ms_compressed"]
+        print(json.dumps(res), flush=True)
+        out.append(res)
+    return {"case": "sweep", "grids": list(grids), "speedups": [r["speedup"] for r in out]}
+
+
+def case_layer(a):
+    """The four projections of one Flash layer (QKV + RoPE, O + residual, FFN
+    up + GELU, FFN down + residual) on --M rows (12,560 = the full 6x34x60
+    sequence, 3,668 = its compressed form), one launch each per iteration:
+    the small case for per-launch DRAM traffic captures."""
+    w = S.WORKLOADS["flash_block_6x34x60"]
+    M, H, A, F = a.M, w.hidden, w.attn_dim, w.ffn
+    g = torch.Generator(device="cuda").manual_seed(6)
+    dims = api.dims_of(w)
+    layers, _ = S.make_weights(w, device="cuda", n_layers=1)
+    l0 = layers[0]
+    xh = torch.randn(M, H, generator=g, device="cuda").bfloat16()
+    xa = torch.randn(M, A, generator=g, device="cuda").bfloat16()
+    resid = torch.randn(M, H, generator=g, device="cuda")
+    pos = torch.randint(0, 60, (M, 3), generator=g, device="cuda", dtype=torch.int32)
+    qkv = torch.empty(M, 3 * A, dtype=torch.bfloat16, device="cuda")
+    u = torch.randn(M, F, generator=g, device="cuda").bfloat16()
+    u_out = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        api.linear(dims, xh, l0["w_qkv"], l0["b_qkv"], L.EPI_QKV_ROPE, pos=pos, out=qkv)
+        api.linear(dims, xa, l0["w_o"], l0["b_o"], L.EPI_RESIDUAL, resid=resid, out=resid)
+        api.linear(dims, xh, l0["w_1"], l0["b_1"], L.EPI_GELU, out=u_out)
+        api.linear(dims, u, l0["w_2"], l0["b_2"], L.EPI_RESIDUAL, resid=resid, out=resid)
+
+    ms = time_it(step, a.iters, a.warmup)
+    fl = 2.0 * M * (4 * A * H + 2 * H * F)
+    return {"case": "layer", "M": M, "ms": ms, "tflops": fl / ms / 1e9,
+            "weight_bytes": 2.0 * (4 * A * H + 2 * H * F)}
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk", "decoder", "generate"])
+    p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk", "decoder", "generate",
+                                    "sweep", "layer"])
     p.add_argument("--n", type=int, default=12560)
     p.add_argument("--heads", type=int, default=56)
     p.add_argument("--M", type=int, default=12560)
@@ -293,6 +383,7 @@ def main():
     p.add_argument("--cut", action="store_true", help="gemm: cut the last wave's tiles along K (fsdit_linear_ws)")
     p.add_argument("--backbone", default="flash_backbone_6x34x60", help="generate: the backbone workload")
     p.add_argument("--rgb8", action="store_true", help="decoder: 8-bit RGB frames (fused colour conversion)")
+    p.add_argument("--grids", default="", help="sweep: comma-separated grids (default 6x17x30,6x34x60,12x34x60)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
@@ -300,7 +391,7 @@ def main():
     L.load()
     res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
            "memory": case_memory, "chunk": case_chunk, "decoder": case_decoder,
-           "generate": case_generate}[a.case](a)
+           "generate": case_generate, "sweep": case_sweep, "layer": case_layer}[a.case](a)
     api.device_error()
     print(json.dumps(res), flush=True)
 

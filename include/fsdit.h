@@ -124,10 +124,12 @@ typedef struct {
  *   grid_t/h/w: the target video grid, rows [0, grid_t*grid_h*grid_w) in
  *     (t,h,w) row-major order (0,0,0 if there is none); control rows follow.
  *   keep_idx [n_keep], near_idx [grid rows]: keep-index map of that grid from
- *     fsdit_build_keep_map (NULL/0: no compression).  The kernels index with
- *     these device arrays as they are: the host checks n_keep against the
- *     grid, but entries that do not come from fsdit_build_keep_map (indices
- *     outside the grid) are undefined behaviour.
+ *     fsdit_build_keep_map (NULL/0: no compression).  The host checks n_keep
+ *     against the grid; the kernels check every entry as they use it (see
+ *     fsdit_gather_rows and fsdit_broadcast_residual): an entry outside the
+ *     grid is never followed, and a map that is not a nearest-kept map is
+ *     reported, through the device error word, as FSDIT_E_SHAPE by
+ *     fsdit_device_error().
  *   pos_thw [n_tokens][3] int32, modality/time_id/out_mask [n_tokens] uint8. */
 typedef struct {
   int n_tokens, n_vrows, n_text, n_audio;
@@ -153,8 +155,9 @@ FSDIT_API const char* fsdit_version(void);
  * instead of trapping.  Returns FSDIT_E_TIMEOUT if a kernel gave up a bounded
  * wait since the word was last cleared, FSDIT_E_SHAPE if the embedding found
  * row tags inconsistent with the sequence's segments (modality or time slot
- * out of place), else FSDIT_OK; a non-zero word is cleared and described in
- * fsdit_last_error(). */
+ * out of place) or the gather / broadcast found a keep_idx / near_idx entry
+ * outside the grid or not forming a nearest-kept map, else FSDIT_OK; a
+ * non-zero word is cleared and described in fsdit_last_error(). */
 FSDIT_API fsdit_status fsdit_device_error(fsdit_stream_t stream);
 
 /* Failure-path check (no fault): launches one thread that waits, through the
@@ -211,7 +214,9 @@ FSDIT_API fsdit_status fsdit_build_keep_map(int T, int H, int W, int32_t* keep_i
  * grid rows keep_idx[c] of x / pos; rows [n_keep, n_keep + n_rows - n_grid)
  * are the non-grid rows n_grid.. n_rows-1 in order (text and audio are never
  * compressed, [PaperDaily] 二).  x, x_c float32 [.., hidden] (device); pos,
- * pos_c int32 [..,3] (device, may both be NULL). */
+ * pos_c int32 [..,3] (device, may both be NULL).  A keep_idx entry outside
+ * [0, n_grid) is not followed: that row of x_c / pos_c is left unwritten and
+ * the device error word is set (fsdit_device_error() returns FSDIT_E_SHAPE). */
 FSDIT_API fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, float* x_c, int32_t* pos_c,
                                const int32_t* keep_idx, int n_keep, int n_grid, int n_rows,
                                int hidden, fsdit_stream_t stream);
@@ -223,7 +228,15 @@ FSDIT_API fsdit_status fsdit_gather_rows(const float* x, const int32_t* pos, flo
  * y_c rows.  The grid is grid_t x grid_h x grid_w (rows [0, T*H*W) of x) with
  * the map of fsdit_build_keep_map (n_keep kept tokens); each kept token's
  * dropped rows lie at +1 / +W / +W+1 of it in its frame.  One launch; out may
- * equal x (every row is read and written by one block only). */
+ * equal x (every row is read and written by one block only).
+ * The kernel checks the map as it uses it: every keep_idx[c] must lie in the
+ * grid with near_idx[keep_idx[c]] == c, and every near_idx[p] must name a
+ * kept token in p's frame at most one row above and one column left of p.
+ * These conditions are exactly those under which every grid row is written
+ * once.  Entries that fail are not followed (no access outside x, y_c, out or
+ * the two maps; the rows they would have produced are left unwritten, which
+ * for out == x means unchanged) and set the device error word, which
+ * fsdit_device_error() reports as FSDIT_E_SHAPE. */
 FSDIT_API fsdit_status fsdit_broadcast_residual(const float* x, const float* y_c, float* out,
                                       const int32_t* keep_idx, const int32_t* near_idx,
                                       int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
@@ -390,13 +403,20 @@ FSDIT_API fsdit_status dit_flow_sample(const fsdit_dims* dims, int n_layers,
  * library (every GPU that loads libfsdit.so holds it until the process
  * exits).  The call allocates nothing: no cudaMalloc, cudaFree or allocating
  * library routine.  Returns FSDIT_E_WORKSPACE, launching nothing, when the
- * block's scratch (fsdit_block_workspace_size) exceeds 32 MiB -- in bf16
- * about 390 tokens at hidden 5376 / 56 heads, about 10,900 at hidden 256 /
- * 2 heads.
+ * block's scratch exceeds 32 MiB.  That scratch is the workspace
+ * dit_block_forward would take: fsdit_block_workspace_size(dims, n, 0) for an
+ * uncompressed block of n rows, and for a compressed block the same function
+ * of its compressed row count n_c = n_keep + (n_tokens - grid rows), i.e.
+ * fsdit_block_workspace_size(dims, n_c, 1).  The largest blocks accepted:
+ *   hidden 5376, 56 x 128 heads, FFN 14336: bf16 387 rows uncompressed,
+ *     310 compressed rows; fp32 194 / 172;
+ *   hidden 2048, 16 x 128 heads, FFN 8192: bf16 1,008 / 808; fp32 508 / 451;
+ *   hidden 256, 2 x 128 heads, FFN 512: bf16 9,362 / 7,262; fp32 5,041 / 4,362.
  *
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  Every call shares the one array and it keeps the last call's
+ * The array's device address is looked up for the current device (once per
+ * device, on the first call with that device current); make that first call
+ * before any stream capture.  `stream` must belong to the current device:
+ * a stream of another device returns FSDIT_E_CUDA, launching nothing.  Every call shares the one array and it keeps the last call's
  * contents (nothing in it needs to start at zero: every buffer is written
  * before it is read).  Calls that overlap on the GPU -- on different streams,
  * or from different threads -- race on it; serialize them. */

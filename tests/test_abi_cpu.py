@@ -155,3 +155,43 @@ def test_linear_ws_rejects_bad_scratch_without_launching(fs):
     d8 = api.make_dims(5376, 42, 14336, L.BF16, proj_fp8=True)
     g = fs.fsdit_linear_fp8_ws
     assert g(C.byref(d8), fake, fake, fake, fake, fake, fake, None, None, 8, 64, 64, 0, fake, need - 1, None) == -6
+
+
+NOALLOC_LIMITS = [  # (hidden, heads, ffn, dtype, largest uncompressed rows, largest compressed rows)
+    (5376, 56, 14336, L.BF16, 387, 310), (5376, 56, 14336, L.F32, 194, 172),
+    (2048, 16, 8192, L.BF16, 1008, 808), (2048, 16, 8192, L.F32, 508, 451),
+    (256, 2, 512, L.BF16, 9362, 7262), (256, 2, 512, L.F32, 5041, 4362),
+]
+
+
+@pytest.mark.parametrize("hidden,heads,ffn,dtype,max_full,max_comp", NOALLOC_LIMITS)
+def test_noalloc_limits_in_the_header_are_the_32_mib_boundaries(fs, hidden, heads, ffn, dtype, max_full, max_comp):
+    # the limits include/fsdit.h lists for dit_block_forward_noalloc: the
+    # largest row counts whose workspace fits the 32 MiB static array; one row
+    # more is refused on the host (FSDIT_E_WORKSPACE) before any CUDA call.
+    # At the limit the host checks pass and the call goes on to look up the
+    # device (no GPU here, so it stops there with another status).
+    d = api.make_dims(hidden, heads, ffn, dtype)
+    lim = 32 << 20
+    assert fs.fsdit_block_workspace_size(C.byref(d), max_full, 0) <= lim
+    assert fs.fsdit_block_workspace_size(C.byref(d), max_full + 1, 0) > lim
+    assert fs.fsdit_block_workspace_size(C.byref(d), max_comp, 1) <= lim
+    assert fs.fsdit_block_workspace_size(C.byref(d), max_comp + 1, 1) > lim
+    fake = C.c_void_p(0x10000)
+    w = L.BlockWeights(*([0x10000] * 10))
+    for compress, limit in ((False, max_full), (True, max_comp)):
+        for extra in (0, 1):
+            tok = L.Tokens()
+            T, H, W = 2, 9, 10                       # 180 grid rows, 60 kept
+            kept = 60 if compress else 180
+            n = limit + extra + (180 - kept)         # rows such that the block's own row count is limit + extra
+            tok.n_tokens, tok.n_vrows, tok.n_text, tok.n_audio = n, 180, n - 180, 0
+            tok.grid_t, tok.grid_h, tok.grid_w = T, H, W
+            tok.pos_thw = 0x10000
+            if compress:
+                tok.keep_idx, tok.n_keep, tok.near_idx = 0x10000, 60, 0x10000
+            st = fs.dit_block_forward_noalloc(C.byref(d), C.byref(w), C.byref(tok), fake, fake, None)
+            if extra:
+                assert st == -6, (compress, L.last_error())
+            else:
+                assert st != -6, (compress, L.last_error())

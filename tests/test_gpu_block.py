@@ -212,3 +212,45 @@ def test_sampler_matches_oracle(dtype):
     assert O.rel_l2(_np(vl), rv) < bound
     assert O.rel_l2(_np(al), ra) < bound
     assert O.rel_l2(_np(vl) - _np(inp["video_lat"]), rv - _np(inp["video_lat"])) < bound
+
+
+def _sampler_vs_oracle(w):
+    layers, io, inp, tags = _setup(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vl, al = inp["video_lat"].to(DEV).clone(), inp["audio_lat"].to(DEV).clone()
+    bb.sample(seq, w.video_clock, w.audio_clock, vl, inp["text_emb"].to(DEV), al)
+    torch.cuda.synchronize()
+    api.device_error()
+    rv, ra = O.flow_sample([S.to_numpy64(l) for l in layers], w.compress, S.to_numpy64(io), _oracle_tok(w, tags),
+                           w.video_clock, w.audio_clock, _np(inp["video_lat"]), _np(inp["text_emb"]),
+                           _np(inp["audio_lat"]), w.heads, w.head_dim)
+    v0, a0 = _np(inp["video_lat"]), _np(inp["audio_lat"])
+    return {"video": O.rel_l2(_np(vl), rv), "audio": O.rel_l2(_np(al), ra),
+            "video_update": O.rel_l2(_np(vl) - v0, rv - v0), "audio_update": O.rel_l2(_np(al) - a0, ra - a0)}
+
+
+@pytest.mark.parametrize("dtype,bound", [("f32", 1e-5), ("bf16", 1e-2)])
+def test_flash_schedule_at_full_depth_matches_oracle(dtype, bound):
+    # the benchmarked schedule itself -- 42 layers, 1-2 full, 3-28 compressed,
+    # 29-42 full ([tokendh] training section, Flash paragraph), 3 evaluations
+    # on the dual clocks -- at small width (hidden 256, 2 x 128 heads), on
+    # the latents and on their total update
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512, grid=(2, 9, 10), n_text=16,
+                 n_audio=8, dtype=dtype)
+    assert w.n_layers == 42 and w.n_evals == 3 and sum(w.compress) == 26
+    err = _sampler_vs_oracle(w)
+    assert max(err.values()) < bound, err
+
+
+@pytest.mark.parametrize("dtype,bound", [("f32", 1e-5), ("bf16", 1e-2)])
+def test_standard_schedule_at_full_depth_matches_oracle(dtype, bound):
+    # the standard model: 50 full layers, 4 evaluations (1 -> 0.2 -> 0.0769 ->
+    # 0.027 -> 0 and 1 -> 0.5 -> 0.25 -> 0.1 -> 0), control frames at a
+    # +16 temporal offset, small width
+    w = S.scaled(S.WORKLOADS["standard_backbone_12x34x60"], hidden=256, heads=2, ffn=512, grid=(2, 9, 10),
+                 control_frames=2, n_text=16, n_audio=8, dtype=dtype)
+    assert w.n_layers == 50 and w.n_evals == 4 and w.n_control > 0
+    err = _sampler_vs_oracle(w)
+    assert max(err.values()) < bound, err
