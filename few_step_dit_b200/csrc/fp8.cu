@@ -2,11 +2,15 @@
 // section 二, third step: low-bit weights and activations, quantization fused
 // next to the normalization).
 //
-// One fp32 scale per row: s = amax / 448 (1 for an all-zero row) and codes
-// E4M3(v * r) with r = 1 / s rounded to fp32 once per row (IEEE reciprocal),
-// round to nearest even, saturating; amax, the reciprocal, the product and the
-// rounding happen in fp32.  Activations are quantized per token, weights per
-// output channel (rows of [N, K]).
+// One fp32 scale per row: s = amax / 448 (fp32 division; 1 for an all-zero
+// row) and codes E4M3(v / s), the exact quotient rounded to nearest with
+// ties to even, saturating at 448.  The quotient is not formed: each value
+// is multiplied by r = fp32(1 / s), and the product t, within about one fp32
+// ulp of the quotient, only picks the E4M3 interval; the side of that
+// interval's midpoint m on which the exact quotient lies is then read off
+// the sign of v - m * s, which one fused multiply-add gives exactly.
+// Activations are quantized per token, weights per output channel (rows of
+// [N, K]).
 
 namespace fsdit {
 namespace q8 {
@@ -51,14 +55,39 @@ template <> __device__ __forceinline__ void load8<bf16>(const bf16* p, float* v)
   }
 }
 
-// 8 codes of v[0..7] * rs (rs: the fp32 reciprocal of the row scale) as one
-// 8-byte word.
-__device__ __forceinline__ uint2 codes8(const float* v, float rs) {
+// The fp32 value whose round-to-nearest-even E4M3 conversion is the code of
+// v / s (s > 0, rs = fp32(1 / s)).  t = |v| rs lies within about one fp32
+// ulp of |v| / s, so the two can fall on different sides only of the
+// midpoint m of the E4M3 interval holding t.  The interval is read from t's
+// bits: above 2^-6 it keeps t's sign, exponent and top three mantissa bits
+// (m sets the fourth and clears the rest); below 2^-6 E4M3 steps by 2^-9,
+// the step of the binade [2^-6, 2^-5), so t is shifted up by 2^-6 and m back
+// down (both exact).  fma(-m, s, |v|) is |v| - m s rounded once, so its sign
+// is that of |v| / s - m (exact for s >= 2^-100: the difference is then a
+// multiple of 2^-149).  The result is m itself for an exact tie (the
+// conversion then picks the even code) or the fp32 neighbour of m on the
+// quotient's side, with v's sign.
+__device__ __forceinline__ float quotient_arg(float v, float s, float rs) {
+  const float av = fabsf(v);
+  const float t = __fmul_rn(av, rs);
+  const bool low = t < 0.015625f;
+  const float tb = low ? __fadd_rn(t, 0.015625f) : t;
+  float m = __uint_as_float((__float_as_uint(tb) & 0xFFF00000u) | 0x00080000u);
+  if (low) m = __fsub_rn(m, 0.015625f);
+  const float r = __fmaf_rn(-m, s, av);
+  const uint32_t mb = __float_as_uint(m);
+  const float a = r > 0.f ? __uint_as_float(mb + 1u) : (r < 0.f ? __uint_as_float(mb - 1u) : m);
+  return copysignf(a, v);
+}
+
+// 8 codes of v[0..7] / s as one 8-byte word (rs: fp32(1 / s)).
+__device__ __forceinline__ uint2 codes8(const float* v, float s, float rs) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = quotient_arg(v[i], s, rs);
   uint2 out;
-  out.x = (uint32_t)e4m3x2(__fmul_rn(v[0], rs), __fmul_rn(v[1], rs)) |
-          ((uint32_t)e4m3x2(__fmul_rn(v[2], rs), __fmul_rn(v[3], rs)) << 16);
-  out.y = (uint32_t)e4m3x2(__fmul_rn(v[4], rs), __fmul_rn(v[5], rs)) |
-          ((uint32_t)e4m3x2(__fmul_rn(v[6], rs), __fmul_rn(v[7], rs)) << 16);
+  out.x = (uint32_t)e4m3x2(a[0], a[1]) | ((uint32_t)e4m3x2(a[2], a[3]) << 16);
+  out.y = (uint32_t)e4m3x2(a[4], a[5]) | ((uint32_t)e4m3x2(a[6], a[7]) << 16);
   return out;
 }
 
@@ -113,7 +142,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
     if (c < cols) {
       float v[8];
       raw[k].get(v);
-      *reinterpret_cast<uint2*>(qr + c) = codes8(v, rs);
+      *reinterpret_cast<uint2*>(qr + c) = codes8(v, sc, rs);
     }
   }
 }
@@ -139,7 +168,7 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const T* __restric
   for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
     float v[8];
     load8<T>(ar + c, v);
-    *reinterpret_cast<uint2*>(qr + c) = codes8(v, rs);
+    *reinterpret_cast<uint2*>(qr + c) = codes8(v, sc, rs);
   }
 }
 
@@ -183,8 +212,8 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const float* __restr
   for (int k = 0; k < RMS_MAXV; ++k) {
     const int i = threadIdx.x + k * 256;
     if (i < h4)
-      qr[i] = (uint32_t)e4m3x2(__fmul_rn(v[k].x, rs), __fmul_rn(v[k].y, rs)) |
-              ((uint32_t)e4m3x2(__fmul_rn(v[k].z, rs), __fmul_rn(v[k].w, rs)) << 16);
+      qr[i] = (uint32_t)e4m3x2(quotient_arg(v[k].x, sc, rs), quotient_arg(v[k].y, sc, rs)) |
+              ((uint32_t)e4m3x2(quotient_arg(v[k].z, sc, rs), quotient_arg(v[k].w, sc, rs)) << 16);
   }
 }
 

@@ -277,8 +277,9 @@ FSDIT_API fsdit_status fsdit_linear(const fsdit_dims* dims, const void* a, const
  * weights and activations, with quantization fused next to the
  * normalization.  Here: FP8 E4M3 (round to nearest even, saturating at 448)
  * with one fp32 scale per row of each quantized operand -- per token for
- * activations, per output channel for weights: s = amax / 448 (1 for an
- * all-zero row), q = E4M3(value / s), amax, division and rounding in fp32.
+ * activations, per output channel for weights: s = amax / 448 rounded to
+ * fp32 (1 for an all-zero row), q = the E4M3 code of the exact quotient
+ * value / s (ties to even; exact for s >= 2^-100).
  * A projection computes (sum_k qa qw) * sa[row] * sw[col] + b on the tcgen05
  * tensor cores (kind::f8f6f4, fp32 accumulation), then its epilogue. */
 

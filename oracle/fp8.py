@@ -14,9 +14,7 @@ below is a reading:
   token for activations, per output channel for weights: s = amax / 448
   (rounded to fp32, as a stored scale is; 1 for an all-zero row) and
   q = E4M3(value / s), the quotient of the fp32 value by the fp32 scale taken
-  in float64 and rounded once to E4M3.  (A kernel may multiply by a rounded
-  reciprocal of s instead of dividing; its codes then differ from these only
-  where the two quotients straddle an E4M3 rounding midpoint, by one step.)
+  in float64 and rounded once to E4M3 (ties to even).
 * Which projections: the four of every block (QKV, O, FFN up, FFN down); the
   input/output embeddings, the time MLP and the heads stay as they are.
 * GEMM: out = (sum_k q_a q_w) * s_a[row] * s_w[col] + bias, then the
