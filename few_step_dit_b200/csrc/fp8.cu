@@ -12,6 +12,8 @@
 // Activations are quantized per token, weights per output channel (rows of
 // [N, K]).
 
+#include <type_traits>
+
 namespace fsdit {
 namespace q8 {
 
@@ -80,15 +82,67 @@ __device__ __forceinline__ float quotient_arg(float v, float s, float rs) {
   return copysignf(a, v);
 }
 
-// 8 codes of v[0..7] / s as one 8-byte word (rs: fp32(1 / s)).
+// Whether the product t = |v| rs (t >= 0) can round to another code than
+// the exact quotient: t lies within 2 ulps of |v| / s, so only a t within 2
+// ulps of an E4M3 midpoint can -- above 2^-6 the midpoints are the values
+// whose low 20 bits are 0x80000 -- or a t below 2^-6, where the step is
+// fixed (checked on the slow path, rare for scaled rows).
+__device__ __forceinline__ bool near_midpoint(float t) {
+  return t < 0.015625f || (__float_as_uint(t) & 0xFFFFFu) - 0x7FFFEu <= 4u;
+}
+
+// 8 codes of v[0..7] / s as one 8-byte word (rs: fp32(1 / s)).  With
+// SCREEN the product decides every code far from a midpoint and only the few
+// others take quotient_arg: the choice for fp32 rows, where about 1e-4 of the
+// values need it.  bf16 rows hold ratios v / amax of two 8-bit significands,
+// which put about 1% of the quotients within an ulp of a midpoint, so nearly
+// every warp would take the second path; they run quotient_arg throughout.
+template <bool SCREEN>
 __device__ __forceinline__ uint2 codes8(const float* v, float s, float rs) {
   float a[8];
+  if (!SCREEN) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) a[i] = quotient_arg(v[i], s, rs);
+    for (int i = 0; i < 8; ++i) a[i] = quotient_arg(v[i], s, rs);
+    uint2 out;
+    out.x = (uint32_t)e4m3x2(a[0], a[1]) | ((uint32_t)e4m3x2(a[2], a[3]) << 16);
+    out.y = (uint32_t)e4m3x2(a[4], a[5]) | ((uint32_t)e4m3x2(a[6], a[7]) << 16);
+    return out;
+  }
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float t = __fmul_rn(fabsf(v[i]), rs);
+    slow |= near_midpoint(t);
+    a[i] = copysignf(t, v[i]);
+  }
+  if (slow) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (near_midpoint(fabsf(a[i]))) a[i] = quotient_arg(v[i], s, rs);
+  }
   uint2 out;
   out.x = (uint32_t)e4m3x2(a[0], a[1]) | ((uint32_t)e4m3x2(a[2], a[3]) << 16);
   out.y = (uint32_t)e4m3x2(a[4], a[5]) | ((uint32_t)e4m3x2(a[6], a[7]) << 16);
   return out;
+}
+
+// 4 codes of v / s as one 32-bit word, the same way.
+__device__ __forceinline__ uint32_t codes4(float4 v, float s, float rs) {
+  const float in[4] = {v.x, v.y, v.z, v.w};
+  float a[4];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float t = __fmul_rn(fabsf(in[i]), rs);
+    slow |= near_midpoint(t);
+    a[i] = copysignf(t, in[i]);
+  }
+  if (slow) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (near_midpoint(fabsf(a[i]))) a[i] = quotient_arg(in[i], s, rs);
+  }
+  return (uint32_t)e4m3x2(a[0], a[1]) | ((uint32_t)e4m3x2(a[2], a[3]) << 16);
 }
 
 // 8 raw input values of a row kept in registers between the amax pass and
@@ -142,7 +196,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
     if (c < cols) {
       float v[8];
       raw[k].get(v);
-      *reinterpret_cast<uint2*>(qr + c) = codes8(v, sc, rs);
+      *reinterpret_cast<uint2*>(qr + c) = codes8<!std::is_same<T, bf16>::value>(v, sc, rs);
     }
   }
 }
@@ -168,7 +222,7 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const T* __restric
   for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
     float v[8];
     load8<T>(ar + c, v);
-    *reinterpret_cast<uint2*>(qr + c) = codes8(v, sc, rs);
+    *reinterpret_cast<uint2*>(qr + c) = codes8<!std::is_same<T, bf16>::value>(v, sc, rs);
   }
 }
 
@@ -212,8 +266,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const float* __restr
   for (int k = 0; k < RMS_MAXV; ++k) {
     const int i = threadIdx.x + k * 256;
     if (i < h4)
-      qr[i] = (uint32_t)e4m3x2(quotient_arg(v[k].x, sc, rs), quotient_arg(v[k].y, sc, rs)) |
-              ((uint32_t)e4m3x2(quotient_arg(v[k].z, sc, rs), quotient_arg(v[k].w, sc, rs)) << 16);
+      qr[i] = codes4(v[k], sc, rs);
   }
 }
 

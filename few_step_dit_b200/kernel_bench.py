@@ -7,7 +7,7 @@ Examples:
   python -m few_step_dit_b200.kernel_bench decoder [--grid 6x34x60] [--fp8]
   python -m few_step_dit_b200.kernel_bench generate   # 3-eval Flash pass + decoder
   python -m few_step_dit_b200.kernel_bench sweep      # compression sweep, 3 grids
-  python -m few_step_dit_b200.kernel_bench layer --M 3668   # one layer's four projections
+  python -m few_step_dit_b200.kernel_bench layer --rows 3668,12560   # one layer's projections + attention
 Inputs are seeded Gaussians; each case prints one JSON line.
 """
 
@@ -337,33 +337,48 @@ def case_sweep(a):
 
 def case_layer(a):
     """The four projections of one Flash layer (QKV + RoPE, O + residual, FFN
-    up + GELU, FFN down + residual) on --M rows (12,560 = the full 6x34x60
-    sequence, 3,668 = its compressed form), one launch each per iteration:
-    the small case for per-launch DRAM traffic captures."""
+    up + GELU, FFN down + residual) and its attention, on each row count of
+    --rows (default: the compressed and full sequences of the three sweep
+    grids), one launch each per iteration: the small case for per-launch
+    ncu captures (DRAM traffic, tensor-pipe activity).  Prints one JSON line
+    per row count."""
     w = S.WORKLOADS["flash_block_6x34x60"]
-    M, H, A, F = a.M, w.hidden, w.attn_dim, w.ffn
+    H, A, F = w.hidden, w.attn_dim, w.ffn
+    rows = [int(v) for v in a.rows.split(",")] if a.rows else [1184, 3380, 3668, 12560, 7016, 24800]
+    Mx = max(rows)
     g = torch.Generator(device="cuda").manual_seed(6)
     dims = api.dims_of(w)
     layers, _ = S.make_weights(w, device="cuda", n_layers=1)
     l0 = layers[0]
-    xh = torch.randn(M, H, generator=g, device="cuda").bfloat16()
-    xa = torch.randn(M, A, generator=g, device="cuda").bfloat16()
-    resid = torch.randn(M, H, generator=g, device="cuda")
-    pos = torch.randint(0, 60, (M, 3), generator=g, device="cuda", dtype=torch.int32)
-    qkv = torch.empty(M, 3 * A, dtype=torch.bfloat16, device="cuda")
-    u = torch.randn(M, F, generator=g, device="cuda").bfloat16()
-    u_out = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+    xh = torch.randn(Mx, H, generator=g, device="cuda").bfloat16()
+    xa = torch.randn(Mx, A, generator=g, device="cuda").bfloat16()
+    resid = torch.randn(Mx, H, generator=g, device="cuda")
+    pos = torch.randint(0, 60, (Mx, 3), generator=g, device="cuda", dtype=torch.int32)
+    qkv = torch.empty(Mx, 3 * A, dtype=torch.bfloat16, device="cuda")
+    att = torch.empty(Mx, A, dtype=torch.bfloat16, device="cuda")
+    u = torch.randn(Mx, F, generator=g, device="cuda").bfloat16()
+    u_out = torch.empty(Mx, F, dtype=torch.bfloat16, device="cuda")
 
-    def step():
-        api.linear(dims, xh, l0["w_qkv"], l0["b_qkv"], L.EPI_QKV_ROPE, pos=pos, out=qkv)
-        api.linear(dims, xa, l0["w_o"], l0["b_o"], L.EPI_RESIDUAL, resid=resid, out=resid)
-        api.linear(dims, xh, l0["w_1"], l0["b_1"], L.EPI_GELU, out=u_out)
-        api.linear(dims, u, l0["w_2"], l0["b_2"], L.EPI_RESIDUAL, resid=resid, out=resid)
+    def step(M):
+        api.linear(dims, xh[:M], l0["w_qkv"], l0["b_qkv"], L.EPI_QKV_ROPE, pos=pos[:M], out=qkv[:M])
+        api.attention(dims, qkv[:M], att[:M])
+        api.linear(dims, xa[:M], l0["w_o"], l0["b_o"], L.EPI_RESIDUAL, resid=resid[:M], out=resid[:M])
+        api.linear(dims, xh[:M], l0["w_1"], l0["b_1"], L.EPI_GELU, out=u_out[:M])
+        api.linear(dims, u[:M], l0["w_2"], l0["b_2"], L.EPI_RESIDUAL, resid=resid[:M], out=resid[:M])
 
-    ms = time_it(step, a.iters, a.warmup)
-    fl = 2.0 * M * (4 * A * H + 2 * H * F)
-    return {"case": "layer", "M": M, "ms": ms, "tflops": fl / ms / 1e9,
-            "weight_bytes": 2.0 * (4 * A * H + 2 * H * F)}
+    for it in range(a.warmup + a.iters):
+        for M in rows:
+            step(M)
+    torch.cuda.synchronize()
+    out = []
+    for M in rows:
+        ms = time_it(lambda: step(M), a.iters, 0)
+        fl = 2.0 * M * (4 * A * H + 2 * H * F) + 4.0 * M * M * A
+        r = {"case": "layer", "M": M, "ms": ms, "tflops": fl / ms / 1e9, "launches": 5,
+             "weight_bytes": 2.0 * (4 * A * H + 2 * H * F)}
+        print(json.dumps(r), flush=True)
+        out.append(r)
+    return {"case": "layer", "rows": rows}
 
 
 def main():
@@ -384,6 +399,7 @@ def main():
     p.add_argument("--backbone", default="flash_backbone_6x34x60", help="generate: the backbone workload")
     p.add_argument("--rgb8", action="store_true", help="decoder: 8-bit RGB frames (fused colour conversion)")
     p.add_argument("--grids", default="", help="sweep: comma-separated grids (default 6x17x30,6x34x60,12x34x60)")
+    p.add_argument("--rows", default="", help="layer: comma-separated row counts")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
