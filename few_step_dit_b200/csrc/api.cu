@@ -229,7 +229,9 @@ fsdit_status launch_linear_fp8(const fsdit_dims* d, const uint8_t* qa, const voi
 fsdit_status launch_attention(const fsdit_dims* d, const void* qkv, void* out, int n, cudaStream_t st) {
   if (n <= 0) return FSDIT_OK;
   ProfScope ps(PC_ATTN, 1, 4.0 * n * (double)n * attn_dim(d), 4.0 * n * (double)attn_dim(d) * dsize(d->dtype), st);
-  if (d->dtype == FSDIT_BF16) return launch_attention_tc(qkv, out, n, d->heads, attn_dim(d), st);
+  if (d->dtype == FSDIT_BF16)
+    return n >= attention_pair_min_rows() ? launch_attention_pair(qkv, out, n, d->heads, attn_dim(d), st)
+                                           : launch_attention_tc(qkv, out, n, d->heads, attn_dim(d), st);
   return launch_attention_simt(FSDIT_F32, qkv, out, n, d->heads, attn_dim(d), st);
 }
 

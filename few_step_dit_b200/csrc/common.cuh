@@ -605,4 +605,8 @@ fsdit_status launch_attention_simt(int dtype, const void* qkv, void* out, int n,
                                    int hidden, cudaStream_t st);
 fsdit_status launch_attention_tc(const void* qkv, void* out, int n, int heads, int attn,
                                  cudaStream_t st);
+// CTA-pair attention for long sequences (attn_pair.cu) and the row count from
+// which launch_attention uses it.
+fsdit_status launch_attention_pair(const void* qkv, void* out, int n, int heads, int attn, cudaStream_t st);
+int attention_pair_min_rows();
 }  // namespace fsdit

@@ -6,6 +6,7 @@
 #include "simt.cu"
 #include "gemm_tc.cu"
 #include "attn_tc.cu"
+#include "attn_pair.cu"
 #include "noalloc.cu"
 #include "history.cu"
 #include "decoder.cu"

@@ -52,7 +52,8 @@ def case_attention(a):
     out = torch.empty(a.n, A, dtype=torch.bfloat16, device="cuda")
     ms = time_it(lambda: api.attention(dims, qkv, out), a.iters, a.warmup)
     fl = 4.0 * a.n * a.n * A
-    return {"case": "attention", "n": a.n, "heads": a.heads, "ms": ms, "tflops": fl / ms / 1e9}
+    kernel = "pair" if a.n >= L.load().fsdit_attention_pair_min_rows() else "single"
+    return {"case": "attention", "n": a.n, "heads": a.heads, "kernel": kernel, "ms": ms, "tflops": fl / ms / 1e9}
 
 
 def case_gemm(a):
@@ -400,11 +401,15 @@ def main():
     p.add_argument("--rgb8", action="store_true", help="decoder: 8-bit RGB frames (fused colour conversion)")
     p.add_argument("--grids", default="", help="sweep: comma-separated grids (default 6x17x30,6x34x60,12x34x60)")
     p.add_argument("--rows", default="", help="layer: comma-separated row counts")
+    p.add_argument("--pair-min-rows", type=int, default=0,
+                   help="attention: rows from which the CTA-pair kernel runs (0: the library default)")
     p.add_argument("--iters", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
     B.build()
-    L.load()
+    lib = L.load()
+    if a.pair_min_rows > 0:
+        L.check("fsdit_set_attention_pair_min_rows", lib.fsdit_set_attention_pair_min_rows(a.pair_min_rows))
     res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
            "memory": case_memory, "chunk": case_chunk, "decoder": case_decoder,
            "generate": case_generate, "sweep": case_sweep, "layer": case_layer}[a.case](a)

@@ -339,6 +339,16 @@ FSDIT_API fsdit_status fsdit_linear_fp8_ws(const fsdit_dims* dims, const uint8_t
 FSDIT_API fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n,
                              fsdit_stream_t stream);
 
+/* Attention kernel choice (bf16).  Sequences of at least `rows` rows run on
+ * the CTA-pair kernel (clusters of two CTAs, 512 queries per cluster, each
+ * CTA staging half of every key and value block); shorter ones on the
+ * single-CTA kernel (256 queries per CTA).  Both compute the same attention;
+ * the threshold is a tuning knob for the whole process (not thread-safe
+ * against concurrent launches).  fsdit_attention_pair_min_rows returns the
+ * current value.  Errors: FSDIT_E_SHAPE for rows < 1. */
+FSDIT_API fsdit_status fsdit_set_attention_pair_min_rows(int rows);
+FSDIT_API int fsdit_attention_pair_min_rows(void);
+
 /* One DiT block.  x_in, x_out float32 [n_tokens, hidden] (device);
  * x_out may equal x_in.  With tok->keep_idx != NULL the block is the Flash
  * compressed block in per-block form: gather the kept grid rows and all
