@@ -1,69 +1,69 @@
 // Joint attention on the sm_100a tensor cores, CTA-pair form for long
 // sequences (bf16 operands, fp32 softmax; same result as tc_attention_kernel).
 //
-// A cluster of two CTAs on neighbouring SMs takes 512 queries of one head as
-// two 256-row pair tiles A and B; CTA rank r holds rows r*128 .. r*128+127 of
-// each.  Every MMA is tcgen05.mma.cta_group::2 (M = 256) issued by one thread
-// of rank 0:
-//   S_t = Q_t K_j^T   N = 128 keys: rank r stages keys r*64 .. r*64+63 of
-//                     block j (K-major), so each CTA loads half of K;
-//   O_t += P_t V_j    N = 128 head columns: rank r stages columns
-//                     r*64 .. r*64+63 of V_j for all 128 keys (MN-major),
-//                     so each CTA loads half of V.
-// Each CTA's TMEM holds S_A, S_B, O_A, O_B for its own 128 rows (512
-// columns).  P is written by the softmax threads into shared memory (the
-// halved K/V stages leave room for P_A and P_B), not over S: once a softmax
-// warp has loaded its S_t(j) row into registers it signals the issuer, which
-// computes S_t(j+1) while the exponentials of block j run.  The tensor pipe
-// then alternates S(j+1) and PV(j) of both tiles with no softmax in between,
-// instead of waiting, per tile, for softmax -> PV -> next S.
+// A cluster of two CTAs on neighbouring SMs takes 256 queries of one head;
+// CTA rank r holds rows r*128 .. r*128+127.  Every MMA is
+// tcgen05.mma.cta_group::2 (M = 256) issued by one thread of rank 0, and both
+// take their A operand from tensor memory, so each SM reads only its half of
+// B from shared memory (64 bytes per cycle at the tensor pipe's rate):
+//   S(j)  = Q K_j^T   A = Q in TMEM (loaded once per CTA); N = 128 keys:
+//                     rank r stages keys r*64 .. r*64+63 of block j (K-major);
+//   O    += P(j) V_j  A = P(j) in TMEM, written over S(j) as bf16; N = 128
+//                     head columns: rank r stages columns r*64 .. r*64+63 of
+//                     V_j for all 128 keys (MN-major).
+// Each CTA's TMEM: S buffers 0 and 1 (128 columns each), O (128), Q (64).
+// S is double-buffered: while the softmax works on S(j), the tensor pipe runs
+// PV(j-1) and S(j+1), so no softmax waits for a matrix product of its own
+// tile and the pipe never waits for a softmax it does not need.  The pair
+// halves every CTA's share of the key/value stream, and the shared memory,
+// free of Q and P, holds deep K and V rings (the copies take several
+// thousand cycles to land).
 //
-// Threads (320 per CTA): warp 0 lane 0 loads Q, K and V with TMA (each CTA
-// its own halves; completion counted on rank 0's barriers); warp 1 allocates
-// TMEM, and on rank 0 lane 0 issues the MMAs; warps 2-5 / 6-9 run the
-// softmax of tile A / B, one thread per query row (TMEM lane): running max
-// and sum in the log2 domain, O rescaled only when a row max grows by more
-// than 8.  Every wait is bounded (see tc_ptx.cuh).
+// Threads (192 per CTA): warp 0 lane 0 loads K and V with TMA (each CTA its
+// own halves; completion counted on rank 0's barriers); warp 1 allocates
+// TMEM and, on rank 0, lane 0 issues the MMAs; warps 2-5 (one per SM
+// sub-partition, each owning its TMEM lane quarter) load Q into TMEM, then
+// run the softmax, one thread per query row: running max and sum in the
+// log2 domain, O rescaled only when a row max grows by more than 8.  Every
+// wait is bounded (see tc_ptx.cuh).
 #include "tc_ptx.cuh"
 
 namespace fsdit {
 namespace attn2 {
 
 constexpr int BQ = 128, BKV = 128, D = 128;
-constexpr int QT_BYTES = 128 * 128 * 2;  // a 128-row Q or P tile: two 64-column swizzled boxes
-constexpr int QT_HALF = QT_BYTES / 2;
-constexpr int KH_BYTES = 64 * 128 * 2;   // this CTA's 64 keys x 128 columns: two 64-column boxes
+constexpr int KH_BYTES = 64 * 128 * 2;  // this CTA's 64 keys x 128 columns: two 64-column boxes
 constexpr int KH_HALF = KH_BYTES / 2;
-constexpr int VH_BYTES = 128 * 64 * 2;   // 128 keys x this CTA's 64 columns: one box
-constexpr int NS = 2;                    // K and V ring stages
-constexpr int THREADS = 320;
-constexpr int OFF_Q = 0;                    // Q_A, Q_B
-constexpr int OFF_P = 2 * QT_BYTES;         // P_A, P_B
-constexpr int OFF_K = 4 * QT_BYTES;         // K stage s at OFF_K + s * KH_BYTES
-constexpr int OFF_V = OFF_K + NS * KH_BYTES;  // V stage s at OFF_V + s * VH_BYTES
+constexpr int VH_BYTES = 128 * 64 * 2;  // 128 keys x this CTA's 64 columns: one box
+constexpr int NS = 6;                   // K and V ring stages
+constexpr int THREADS = 192;
+constexpr int SOFTMAX_WARPS = 4;
+constexpr int OFF_K = 0;                      // K stage s at OFF_K + s * KH_BYTES
+constexpr int OFF_V = NS * KH_BYTES;          // V stage s at OFF_V + s * VH_BYTES
 constexpr int OFF_BAR = OFF_V + NS * VH_BYTES;
-// barriers; the FULL ones and S_FREE / P_FULL are waited on in rank 0 only
 enum {
-  B_QFULL = 0,
-  B_KFULL = 1,
-  B_VFULL = B_KFULL + NS,
-  B_KEMPTY = B_VFULL + NS,
-  B_VEMPTY = B_KEMPTY + NS,
-  B_SFULL = B_VEMPTY + NS,  // per tile, in both CTAs: S_t ready in TMEM
-  B_SFREE = B_SFULL + 2,    // per tile, rank 0: both CTAs' S_t rows are in registers
-  B_PFULL = B_SFREE + 2,    // per tile, rank 0: both CTAs' P_t written (and O_t rescaled)
-  B_PFREE = B_PFULL + 2,    // per tile, in both CTAs: PV_t done (P_t free, O_t stable)
-  B_ODONE = B_PFREE + 2,    // per tile, in both CTAs: the last PV_t done
-  B_DRAIN = B_ODONE + 2,
+  B_KFULL = 0,                // rank 0: both CTAs' K halves landed
+  B_VFULL = B_KFULL + NS,     // rank 0: both CTAs' V halves landed
+  B_KEMPTY = B_VFULL + NS,    // both CTAs: the S MMA reading the stage is done
+  B_VEMPTY = B_KEMPTY + NS,   // both CTAs: the PV MMA reading the stage is done
+  B_QREADY = B_VEMPTY + NS,   // rank 0: both CTAs' Q rows are in TMEM
+  B_SFULL = B_QREADY + 1,     // both CTAs, per S buffer: S ready
+  B_PFULL = B_SFULL + 2,      // rank 0: both CTAs' P(j) written (and O rescaled)
+  B_PFREE = B_PFULL + 1,      // both CTAs: PV(j) done (O stable)
+  B_ODONE = B_PFREE + 1,      // both CTAs: the last PV done
+  B_DRAIN = B_ODONE + 1,
   NUM_BARS = B_DRAIN + 1
 };
 constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0;    // S buffer b at COL_S + 128 b
+constexpr uint32_t COL_O = 256;
+constexpr uint32_t COL_Q = 384;  // Q as packed bf16 pairs (64 columns)
 constexpr uint32_t IDESC_S = ptx::idesc_bf16(2 * BQ, BKV, 0);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16(2 * BQ, D, 1);
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-constexpr int SOFTMAX_WARPS = 8;           // arrivals per tile barrier: 4 warps x 2 CTAs
+constexpr int ARRIVALS = 2 * SOFTMAX_WARPS;  // per phase of the softmax-to-issuer barriers: both CTAs
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -115,22 +115,27 @@ __device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
   return r;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+// Pair MMA with A in tensor memory (each CTA's TMEM holds its 128 rows), B
+// in shared memory (each CTA its half of N), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (the tensor core's operand reads), including reads issued by the
-// peer CTA's MMA thread after the cluster-scope barrier arrive that follows.
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
 struct Args {
-  int n, heads, attn;  // attn = heads * 128
-  bf16* out;           // [n, attn]
-  float scale_log2;    // log2(e) / sqrt(128)
+  int n, heads, attn;   // attn = heads * 128
+  const bf16* qkv;      // [n, 3 attn]
+  bf16* out;            // [n, attn]
+  float scale_log2;     // log2(e) / sqrt(128)
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
-    tc_attention_pair_kernel(const __grid_constant__ CUtensorMap tmQV, const __grid_constant__ CUtensorMap tmK,
+    tc_attention_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                              const Args args) {
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
@@ -145,32 +150,30 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int head = blockIdx.y;
-  const int q0 = (int)(blockIdx.x >> 1) * 4 * BQ;  // first query of the cluster's 512
+  const int q0 = (int)(blockIdx.x >> 1) * 2 * BQ + (int)rank * BQ;  // this CTA's first query
   const int n = args.n;
   const int nkv = (n + BKV - 1) / BKV;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_QFULL), 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_KEMPTY + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(B_SFULL + t), 1);
-      mbar_init(bar(B_SFREE + t), SOFTMAX_WARPS);
-      mbar_init(bar(B_PFULL + t), SOFTMAX_WARPS);
-      mbar_init(bar(B_PFREE + t), 1);
-      mbar_init(bar(B_ODONE + t), 1);
-    }
+    mbar_init(bar(B_QREADY), ARRIVALS);
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_SFULL + 1), 1);
+    mbar_init(bar(B_PFULL), ARRIVALS);
+    mbar_init(bar(B_PFREE), 1);
+    mbar_init(bar(B_ODONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmQV);
     prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
@@ -185,43 +188,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // producer: Q once, then K(j+1) before V(j) (K is needed a block earlier)
-      const uint32_t qfull0 = peer_addr(bar(B_QFULL), 0u);
+      // producer: K(i) and V(i) halves into their rings, K first (needed a block earlier)
       const uint32_t kfull0 = peer_addr(bar(B_KFULL), 0u), vfull0 = peer_addr(bar(B_VFULL), 0u);
       bool ok = true;
-      if (rank == 0) mbar_expect_tx(bar(B_QFULL), 2 * 2 * QT_BYTES);
-      for (int t = 0; t < 2; ++t) {
-        const int row = q0 + t * 2 * BQ + (int)rank * BQ;
-        tma_load_2d_pair(base + OFF_Q + t * QT_BYTES, &tmQV, cq, row, qfull0);
-        tma_load_2d_pair(base + OFF_Q + t * QT_BYTES + QT_HALF, &tmQV, cq + 64, row, qfull0);
-      }
       int last_k = -1, last_v = -1;
-      auto load_k = [&](int i) -> bool {
+      for (int i = 0; i < nkv && ok; ++i) {
         const int s = i % NS;
         const uint32_t ph = (uint32_t)(i / NS) & 1u;
-        if (!mbar_wait(bar(B_KEMPTY + s), ph ^ 1u, abort_flag)) return false;
+        if (!mbar_wait(bar(B_KEMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
         if (rank == 0) mbar_expect_tx(bar(B_KFULL + s), 2 * KH_BYTES);
-        const uint32_t dst = base + OFF_K + s * KH_BYTES;
-        const int row = i * BKV + (int)rank * 64;
-        tma_load_2d_pair(dst, &tmK, ck, row, kfull0 + 8u * (uint32_t)s);
-        tma_load_2d_pair(dst + KH_HALF, &tmK, ck + 64, row, kfull0 + 8u * (uint32_t)s);
+        const uint32_t dk = base + OFF_K + s * KH_BYTES;
+        const int krow = i * BKV + (int)rank * 64;
+        tma_load_2d_pair(dk, &tmK, ck, krow, kfull0 + 8u * (uint32_t)s);
+        tma_load_2d_pair(dk + KH_HALF, &tmK, ck + 64, krow, kfull0 + 8u * (uint32_t)s);
         last_k = i;
-        return true;
-      };
-      auto load_v = [&](int i) -> bool {
-        const int s = i % NS;
-        const uint32_t ph = (uint32_t)(i / NS) & 1u;
-        if (!mbar_wait(bar(B_VEMPTY + s), ph ^ 1u, abort_flag)) return false;
+        if (!mbar_wait(bar(B_VEMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
         if (rank == 0) mbar_expect_tx(bar(B_VFULL + s), 2 * VH_BYTES);
-        tma_load_2d_pair(base + OFF_V + s * VH_BYTES, &tmQV, cv + (int)rank * 64, i * BKV,
-                         vfull0 + 8u * (uint32_t)s);
+        tma_load_2d_pair(base + OFF_V + s * VH_BYTES, &tmV, cv + (int)rank * 64, i * BKV, vfull0 + 8u * (uint32_t)s);
         last_v = i;
-        return true;
-      };
-      if (nkv > 0) ok = load_k(0);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv && !load_k(j + 1)) { ok = false; break; }
-        if (!load_v(j)) { ok = false; break; }
       }
       // on abort, let the newest copies land before the CTA can exit (rank 1
       // cannot observe rank 0's barriers; its copies finish within microseconds)
@@ -242,63 +226,50 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit_pair(bar(b));
         tc_commit_pair(peer_bar0 + 8u * (uint32_t)b);
       };
-      // S_t(j) = Q_t K_j^T into TMEM columns 128t (each CTA: its 128 rows, all 128 keys)
-      auto issue_s = [&](int t, int j) {
-        const uint32_t sk = base + OFF_K + (j % NS) * KH_BYTES;
-        const uint32_t sq = base + OFF_Q + t * QT_BYTES;
+      // descriptors: the address field holds (address >> 4), so a stage or a
+      // K step further is the base descriptor plus (offset >> 4)
+      const uint64_t dk = sw128_desc(base + OFF_K, 16, 1024), dv = sw128_desc(base + OFF_V, VH_BYTES, 1024);
+      // S(j) = Q K_j^T into S buffer j % 2
+      auto issue_s = [&](int j) {
+        const uint64_t bk = dk + (uint64_t)(((j % NS) * KH_BYTES) >> 4);
+        const uint32_t d = tmem + COL_S + (uint32_t)((j & 1) * BKV);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t oq = (uint32_t)((k >> 2) * QT_HALF + (k & 3) * 32);
-          const uint32_t ok_ = (uint32_t)((k >> 2) * KH_HALF + (k & 3) * 32);
-          mma_bf16_ss_pair(tmem + (uint32_t)(t * BKV), sw128_desc(sq + oq, 16, 1024), sw128_desc(sk + ok_, 16, 1024),
-                           IDESC_S, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < D / 16; ++k)
+          mma_bf16_ts_pair(d, tmem + COL_Q + (uint32_t)(k * 8),
+                           bk + (uint64_t)(((k >> 2) * KH_HALF + (k & 3) * 32) >> 4), IDESC_S, k > 0 ? 1u : 0u);
       };
-      // O_t += P_t(j) V_j (P_t in shared memory, K-major; V MN-major)
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t sp = base + OFF_P + t * QT_BYTES;
-        const uint32_t sv = base + OFF_V + (j % NS) * VH_BYTES;
+      // O += P(j) V_j, P(j) in the first 64 columns of S buffer j % 2
+      auto issue_pv = [&](int j) {
+        const uint64_t bv = dv + (uint64_t)(((j % NS) * VH_BYTES) >> 4);
+        const uint32_t p = tmem + COL_S + (uint32_t)((j & 1) * BKV);
 #pragma unroll
-        for (int k = 0; k < BKV / 16; ++k) {
-          const uint32_t op = (uint32_t)((k >> 2) * QT_HALF + (k & 3) * 32);
-          mma_bf16_ss_pair(tmem + 256u + (uint32_t)(t * D), sw128_desc(sp + op, 16, 1024),
-                           sw128_desc(sv + (uint32_t)(k * 2048), VH_BYTES, 1024), IDESC_PV,
+        for (int k = 0; k < BKV / 16; ++k)
+          mma_bf16_ts_pair(tmem + COL_O, p + (uint32_t)(k * 8), bv + (uint64_t)((k * 2048) >> 4), IDESC_PV,
                            (j > 0 || k > 0) ? 1u : 0u);
-        }
       };
-      bool ok = nkv > 0 && mbar_wait(bar(B_QFULL), 0, abort_flag);
-      if (ok) ok = mbar_wait(bar(B_KFULL), 0, abort_flag);
+      auto s_step = [&](int j) -> bool {  // K(j) landed -> S(j)
+        if (!mbar_wait(bar(B_KFULL + j % NS), (uint32_t)(j / NS) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        issue_s(j);
+        commit_both(B_SFULL + (j & 1));
+        commit_both(B_KEMPTY + j % NS);
+        return true;
+      };
+      bool ok = nkv > 0 && mbar_wait(bar(B_QREADY), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          issue_s(t, 0);
-          commit_both(B_SFULL + t);
-        }
-        commit_both(B_KEMPTY);
+        ok = s_step(0);
       }
+      if (ok && nkv > 1) ok = s_step(1);
       for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) % NS;
-          if (!mbar_wait(bar(B_KFULL + s1), (uint32_t)((j + 1) / NS) & 1u, abort_flag)) { ok = false; break; }
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (!mbar_wait_cluster(bar(B_SFREE + t), (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(t, j + 1);
-            commit_both(B_SFULL + t);
-          }
-          if (!ok) break;
-          commit_both(B_KEMPTY + s1);
-        }
-        const int s = j % NS;
-        if (!mbar_wait(bar(B_VFULL + s), (uint32_t)(j / NS) & 1u, abort_flag)) { ok = false; break; }
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait_cluster(bar(B_PFULL + t), (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, j);
-          commit_both(j + 1 < nkv ? B_PFREE + t : B_ODONE + t);
-        }
-        if (!ok) break;
-        commit_both(B_VEMPTY + s);
+        if (!mbar_wait(bar(B_VFULL + j % NS), (uint32_t)(j / NS) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(B_PFULL), (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(j);
+        commit_both(j + 1 < nkv ? B_PFREE : B_ODONE);
+        commit_both(B_VEMPTY + j % NS);
+        // S buffer j % 2 is free once PV(j) has read P(j) (the pipe runs in issue order)
+        if (j + 2 < nkv && !s_step(j + 2)) { ok = false; break; }
       }
       // every MMA this thread issued has completed (and stopped reading both
       // CTAs' shared memory) once DRAIN flips
@@ -306,34 +277,48 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait(bar(B_DRAIN), 0, nullptr);
     }
   } else {
-    // softmax: tile t, thread <-> query row r of this CTA's half of the tile (TMEM lane r)
-    const int t = (warp - 2) >> 2;
+    // softmax warps 2-5: warp w owns TMEM lanes 32 (w % 4) .. +31; thread <-> query row r
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    const uint32_t s_col = (uint32_t)(t * BKV);
-    const uint32_t o_col = 256u + (uint32_t)(t * D);
-    const uint32_t p_row = base + OFF_P + (uint32_t)(t * QT_BYTES) + (uint32_t)(r * 128);
-    const uint32_t swz = (uint32_t)(r & 7);
-    const uint32_t sfree0 = peer_addr(bar(B_SFREE + t), 0u), pfull0 = peer_addr(bar(B_PFULL + t), 0u);
+    const uint32_t qready0 = peer_addr(bar(B_QREADY), 0u), pfull0 = peer_addr(bar(B_PFULL), 0u);
+    const int row = q0 + r;
+    // Q row into TMEM as packed bf16 pairs (the A-operand layout of the S MMA); rows past n are 0
+    {
+      uint32_t qv[64];
+      if (row < n) {
+        const uint4* src = reinterpret_cast<const uint4*>(args.qkv + (size_t)row * 3 * args.attn + cq);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 u = __ldg(src + i);
+          qv[4 * i] = u.x;
+          qv[4 * i + 1] = u.y;
+          qv[4 * i + 2] = u.z;
+          qv[4 * i + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) qv[i] = 0u;
+      }
+      tmem_st64(tmem + lane_addr + COL_Q, qv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(qready0);
+    }
     const float sl2 = args.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // one lane waits on a barrier of this CTA, the warp follows
     auto warp_wait = [&](int b, uint32_t parity) -> bool {
       int w_ok = 1;
       if (lane == 0) w_ok = mbar_wait(bar(b), parity, abort_flag) ? 1 : 0;
       return __shfl_sync(0xffffffffu, w_ok, 0) != 0;
     };
     for (int j = 0; j < nkv; ++j) {
-      if (!warp_wait(B_SFULL + t, (uint32_t)j & 1u)) { ok = false; break; }
+      const uint32_t s_col = COL_S + (uint32_t)((j & 1) * BKV);
+      if (!warp_wait(B_SFULL + (j & 1), (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
       tc_fence_after();
       float s[BKV];
       tmem_ld128(tmem + lane_addr + s_col, s);
-      // this warp's S rows are in registers: the issuer may overwrite S_t
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(sfree0);
       const int valid = n - j * BKV;  // keys past n are masked
       if (valid < BKV) {
 #pragma unroll
@@ -344,15 +329,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool grow = m_cand > m + RESCALE_THRESHOLD;
       const float m_new = grow ? m_cand : m;
       const float corr = grow ? ex2(m - m_new) : 1.0f;
-      bool pv_done = j == 0;  // PV_t(j-1) has finished with P_t and O_t
+      // O is stable once PV(j-1) is done; only a rescale has to wait for it
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        if (!warp_wait(B_PFREE + t, (uint32_t)(j - 1) & 1u)) { ok = false; break; }
-        pv_done = true;
+        if (!warp_wait(B_PFREE, (uint32_t)(j - 1) & 1u)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          const uint32_t ta = tmem + lane_addr + o_col + (uint32_t)(c * 32);
+          const uint32_t ta = tmem + lane_addr + COL_O + (uint32_t)(c * 32);
           tmem_ld32(ta, o);
           uint32_t u[32];
 #pragma unroll
@@ -371,34 +355,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2(p0, p1));
         pk[c >> 1] = pack_bf16(p0, p1);
       }
-      if (!pv_done && !warp_wait(B_PFREE + t, (uint32_t)(j - 1) & 1u)) { ok = false; break; }
-      // P_t row r: keys 64b .. 64b+63 in box b, 16-byte chunk cc at (cc ^ (r & 7)) (128-byte swizzle)
-#pragma unroll
-      for (int b = 0; b < 2; ++b) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint32_t* v = pk + b * 32 + cc * 4;
-          st_shared_v4(p_row + (uint32_t)(b * QT_HALF) + (((uint32_t)cc ^ swz) << 4), v[0], v[1], v[2], v[3]);
-        }
-      }
-      fence_proxy_async_all();
+      // P(j) over the first 64 columns of its S buffer
+      tmem_st64(tmem + lane_addr + s_col, pk);
       float a0, a1;
       f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
       l = l * corr + (a0 + a1);
       m = m_new;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(pfull0);
+      if (lane == 0) mbar_arrive_remote(pfull0);
     }
-    if (ok && nkv > 0 && warp_wait(B_ODONE + t, 0u)) {
+    if (ok && nkv > 0 && warp_wait(B_ODONE, 0u)) {
       tc_fence_after();
-      const int row = q0 + t * 2 * BQ + (int)rank * BQ + r;
       const float inv = 1.0f / l;
       bf16* orow = args.out + (size_t)row * args.attn + head * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tmem_ld32(tmem + lane_addr + o_col + (uint32_t)(c * 32), o);
+        tmem_ld32(tmem + lane_addr + COL_O + (uint32_t)(c * 32), o);
         if (row < n) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
@@ -427,6 +401,10 @@ int attention_pair_min_rows() { return g_attn_pair_min_rows; }
 
 fsdit_status launch_attention_pair(const void* qkv, void* out, int n, int heads, int attn_w, cudaStream_t st) {
   using namespace attn2;
+  if (((uintptr_t)qkv & 15u) != 0) {
+    set_error("attention: qkv must be 16-byte aligned");
+    return FSDIT_E_ALIGN;
+  }
   static PerDevice<cudaError_t> attr;
   const cudaError_t attr_err = attr.get(
       [] {
@@ -435,16 +413,17 @@ fsdit_status launch_attention_pair(const void* qkv, void* out, int n, int heads,
       },
       cudaErrorInvalidDevice);
   if (attr_err != cudaSuccess) return cuda_check(attr_err, "cudaFuncSetAttribute(tc_attention_pair_kernel)");
-  CUtensorMap tmQV, tmK;
-  FS_TRY(make_tmap_bf16(&tmQV, qkv, (uint64_t)n, (uint64_t)3 * attn_w, (uint64_t)3 * attn_w, 128, 64));
+  CUtensorMap tmK, tmV;
   FS_TRY(make_tmap_bf16(&tmK, qkv, (uint64_t)n, (uint64_t)3 * attn_w, (uint64_t)3 * attn_w, 64, 64));
+  FS_TRY(make_tmap_bf16(&tmV, qkv, (uint64_t)n, (uint64_t)3 * attn_w, (uint64_t)3 * attn_w, 128, 64));
   Args a;
   a.n = n;
   a.heads = heads;
   a.attn = attn_w;
+  a.qkv = reinterpret_cast<const bf16*>(qkv);
   a.out = reinterpret_cast<bf16*>(out);
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  const int nqb = (n + 4 * BQ - 1) / (4 * BQ);
+  const int nqb = (n + 2 * BQ - 1) / (2 * BQ);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -457,7 +436,7 @@ fsdit_status launch_attention_pair(const void* qkv, void* out, int n, int heads,
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, tc_attention_pair_kernel, tmQV, tmK, a), "tc_attention_pair_kernel");
+  return cuda_check(cudaLaunchKernelEx(&cfg, tc_attention_pair_kernel, tmK, tmV, a), "tc_attention_pair_kernel");
 }
 
 }  // namespace fsdit

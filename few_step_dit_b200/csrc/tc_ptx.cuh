@@ -218,6 +218,15 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
+// Arrive on an mbarrier of either CTA of the cluster with CTA-scope release:
+// orders only this CTA's prior accesses (a cluster-scope release waits for
+// every prior write of the thread to become visible cluster-wide, hundreds of
+// cycles).  For signals whose data stays in the arriving CTA -- its TMEM rows
+// read, its own shared memory written for its own tensor core (after a proxy
+// fence).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
