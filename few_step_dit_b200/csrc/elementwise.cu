@@ -272,9 +272,28 @@ __global__ void __launch_bounds__(256) embed_kernel(
     s_t[threadIdx.x] = t;
   }
   if (kind == 1) {
-    for (int i = threadIdx.x; i < EMB_RB * KMAX; i += blockDim.x) {
-      const int rr = i % EMB_RB, kk = i / EMB_RB;  // consecutive threads: consecutive rows (no bank conflict)
-      s_latT[kk][rr] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
+    // the block's rows are nr * K contiguous floats, transposed into the
+    // channel-major stage; channels past K and rows past nr are zero
+    if (K % 4 == 0) {  // 16-byte loads (the rows start 16-byte aligned: rb0 * K * 4 = 512 * K)
+      const float4* src = reinterpret_cast<const float4*>(lat + (size_t)rb0 * K);
+      const int n4 = nr * K / 4;
+      for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+        const float4 v = __ldg(src + i);
+        const int e = 4 * i, rr = e / K, kk = e - rr * K;  // the 4 values share a row
+        s_latT[kk][rr] = v.x;
+        s_latT[kk + 1][rr] = v.y;
+        s_latT[kk + 2][rr] = v.z;
+        s_latT[kk + 3][rr] = v.w;
+      }
+      for (int i = threadIdx.x; i < EMB_RB * KMAX; i += blockDim.x) {
+        const int rr = i % EMB_RB, kk = i / EMB_RB;
+        if (rr >= nr || kk >= K) s_latT[kk][rr] = 0.f;
+      }
+    } else {
+      for (int i = threadIdx.x; i < EMB_RB * KMAX; i += blockDim.x) {
+        const int rr = i % EMB_RB, kk = i / EMB_RB;  // consecutive threads: consecutive rows (no bank conflict)
+        s_latT[kk][rr] = (rr < nr && kk < K) ? lat[(size_t)(rb0 + rr) * K + kk] : 0.f;
+      }
     }
   }
   if (tagged) {
