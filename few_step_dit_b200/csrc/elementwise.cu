@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(256) embed_kernel(
   __shared__ __align__(16) float s_latT[KMAX][EMB_RB];  // channel-major: rows j..j+3 of channel k are one float4
   __shared__ float s_mod[4][EMB_CB];
   __shared__ float s_temb[EMB_MAXT][EMB_CB];
-  __shared__ int s_m[EMB_RB], s_t[EMB_RB];
+  __shared__ __align__(16) int s_mt[EMB_RB];  // modality | time slot << 8 of each row
   const int rb0 = blockIdx.x * EMB_RB;
   const int nr = min(EMB_RB, rows - rb0);
   const int c = blockIdx.y * EMB_CB + threadIdx.x;
@@ -268,8 +268,7 @@ __global__ void __launch_bounds__(256) embed_kernel(
         t = 0;
       }
     }
-    s_m[threadIdx.x] = m;
-    s_t[threadIdx.x] = t;
+    s_mt[threadIdx.x] = m | (t << 8);
   }
   if (kind == 1) {
     // the block's rows are nr * K contiguous floats, transposed into the
@@ -311,7 +310,12 @@ __global__ void __launch_bounds__(256) embed_kernel(
       wd[k] = emb_pair(wv, wv);
     }
     const float bias = ld_f32<TW>(b_in + c);
-    for (int j = 0; j < nr; j += 4) {  // rows past nr are zero in s_latT and not stored
+    // the added embedding of a row depends only on its (modality, time slot),
+    // the same for nearly every row of a segment: keep the last pair's sum
+    int last_mt = -1;
+    float add = 0.f;
+    float* xp = x + (size_t)(row0 + rb0) * hidden + c;
+    for (int j = 0; j < nr; j += 4, xp += 4 * (size_t)hidden) {  // rows past nr are zero in s_latT, not stored
       emb_f2 a01 = emb_pair(bias, bias), a23 = emb_pair(bias, bias);
 #pragma unroll
       for (int k = 0; k < KMAX; ++k) {
@@ -322,18 +326,23 @@ __global__ void __launch_bounds__(256) embed_kernel(
       float v[4];
       emb_split(a01, v[0], v[1]);
       emb_split(a23, v[2], v[3]);
+      int4 mt = make_int4(0, 0, 0, 0);
+      if (tagged) mt = *reinterpret_cast<const int4*>(&s_mt[j]);
+      const int mts[4] = {mt.x, mt.y, mt.z, mt.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         if (j + u >= nr) break;
-        float acc = v[u];
-        if (tagged) acc += s_mod[s_m[j + u]][threadIdx.x] + s_temb[s_t[j + u]][threadIdx.x];
-        x[(size_t)(row0 + rb0 + j + u) * hidden + c] = acc;
+        if (tagged && mts[u] != last_mt) {  // uniform across the block: the row's tags
+          last_mt = mts[u];
+          add = s_mod[last_mt & 0xFF][threadIdx.x] + s_temb[last_mt >> 8][threadIdx.x];
+        }
+        xp[(size_t)u * hidden] = v[u] + add;
       }
     }
   } else {
     for (int j = 0; j < nr; ++j) {
       float acc = text_proj[(size_t)(rb0 + j) * hidden + c];
-      if (tagged) acc += s_mod[s_m[j]][threadIdx.x] + s_temb[s_t[j]][threadIdx.x];
+      if (tagged) acc += s_mod[s_mt[j] & 0xFF][threadIdx.x] + s_temb[s_mt[j] >> 8][threadIdx.x];
       x[(size_t)(row0 + rb0 + j) * hidden + c] = acc;
     }
   }

@@ -336,6 +336,22 @@ def case_sweep(a):
     return {"case": "sweep", "grids": list(grids), "speedups": [r["speedup"] for r in out]}
 
 
+def case_embed(a):
+    """The backbone's input side alone: a stack of zero layers (timestep MLP,
+    text projection, the three embedding launches, final RMSNorm and heads) on
+    the 6x34x60 sequence, replayed from a CUDA graph, plus a per-class profile:
+    the small case for captures of the embedding kernel."""
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], n_layers=0, compress=())
+    _, io = S.make_weights(w, device="cuda", n_layers=0)
+    bb = api.Backbone(api.dims_of(w), [], api.IOWeights(io), ())
+    seq = api.Sequence.from_workload(w, S.pack_tokens(w), "cuda", compress=False)
+    inp = S.make_inputs(w, device="cuda")
+    table = [0.0, w.video_clock[0], w.audio_clock[0]]
+    step = lambda: bb.forward(seq, table, inp["video_lat"], inp["text_emb"], inp["audio_lat"])  # noqa: E731
+    ms = _graph_ms(step, a)
+    return {"case": "embed", "tokens": w.n_tokens, "ms": ms, "classes": _profile(step)}
+
+
 def case_layer(a):
     """The four projections of one Flash layer (QKV + RoPE, O + residual, FFN
     up + GELU, FFN down + residual) and its attention, on each row count of
@@ -385,7 +401,7 @@ def case_layer(a):
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("case", choices=["attention", "gemm", "block", "memory", "chunk", "decoder", "generate",
-                                    "sweep", "layer"])
+                                    "sweep", "layer", "embed"])
     p.add_argument("--n", type=int, default=12560)
     p.add_argument("--heads", type=int, default=56)
     p.add_argument("--M", type=int, default=12560)
@@ -412,7 +428,7 @@ def main():
         L.check("fsdit_set_attention_pair_min_rows", lib.fsdit_set_attention_pair_min_rows(a.pair_min_rows))
     res = {"attention": case_attention, "gemm": case_gemm, "block": case_block,
            "memory": case_memory, "chunk": case_chunk, "decoder": case_decoder,
-           "generate": case_generate, "sweep": case_sweep, "layer": case_layer}[a.case](a)
+           "generate": case_generate, "sweep": case_sweep, "layer": case_layer, "embed": case_embed}[a.case](a)
     api.device_error()
     print(json.dumps(res), flush=True)
 
