@@ -17,7 +17,7 @@ static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "ge
                                            "broadcast",     "embed",         "time_mlp",  "heads",
                                            "euler",         "keep_map",  "rope_table", "history_gather",
                                            "quantize",      "gemm_fp8_qkv_rope", "gemm_fp8_residual",
-                                           "gemm_fp8_gelu", "grid_positions", "pixel_head"};
+                                           "gemm_fp8_gelu", "grid_positions", "pixel_head", "rms_rstd"};
 struct Prof {
   bool on = false;
   int used = 0;
@@ -65,6 +65,7 @@ fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_
 fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
                               const int32_t* near_idx, int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
                               int hidden, cudaStream_t st);
+fsdit_status launch_rstd(const float* ss, int parts, int rows, int hidden, float eps, float* rstd, cudaStream_t st);
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
                                  cudaStream_t st);
 fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
@@ -256,7 +257,23 @@ struct BlockWs {  // every buffer null until a carve sets it
   float2* rope_c = nullptr;  // stack only: table of the compressed rows
   uint8_t* q8 = nullptr;     // FP8 projections: [n, max(hidden, attn, ffn)] E4M3 operand
   float* sa = nullptr;       //                  [n] its row scales
+  float* ss = nullptr;       // RMSNorm after the GEMM: [n, hidden/128] sums of squares per column group
+  float* rstd = nullptr;     //                         [n] 1/rms per row
 };
+
+// Blocks run back to back (stack, decoder) apply each RMSNorm after the GEMM
+// that consumes it: the residual epilogue before the norm writes bf16(x * g)
+// and per-group sums of squares, and the consuming GEMM scales its rows by
+// 1/rms.  bf16 tensor-core projections with hidden % 128 == 0 only.
+static bool norm_after_gemm(const fsdit_dims* d) {
+  return d->dtype == FSDIT_BF16 && !d->proj_fp8 && d->hidden % 128 == 0;
+}
+
+static void carve_norm(Carve& c, const fsdit_dims* d, int n_rows, BlockWs& w) {
+  if (!norm_after_gemm(d)) return;
+  w.ss = (float*)c.take((size_t)n_rows * (d->hidden / 128) * 4);
+  w.rstd = (float*)c.take((size_t)n_rows * 4);
+}
 
 static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, bool compressed) {
   BlockWs w;
@@ -323,21 +340,54 @@ static fsdit_status block_body_fp8(const fsdit_dims* d, const fsdit_block_weight
   return FSDIT_OK;
 }
 
+// in_ready: ws.xn already holds bf16(x_in * g_attn) and ws.ss its sums of
+// squares (the previous block's FFN-down epilogue wrote them).  g_next: the
+// gain of the norm that follows this block on the same rows, or null; the
+// FFN-down epilogue then prepares it and *out_ready is set.
 static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w, float* x_in, float* x_out,
-                               const int32_t* pos, const float2* rope, int n, const BlockWs& ws, cudaStream_t st) {
+                               const int32_t* pos, const float2* rope, int n, const BlockWs& ws, cudaStream_t st,
+                               bool in_ready = false, const void* g_next = nullptr, bool* out_ready = nullptr) {
+  if (out_ready) *out_ready = false;
   if (d->proj_fp8) return block_body_fp8(d, w, x_in, x_out, pos, rope, n, ws, st);
   const int H = d->hidden, F = d->ffn, A = attn_dim(d);
-  FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
+  const bool fuse = ws.ss != nullptr && ws.rstd != nullptr;
+  auto produce = [&](EpiParams e, void* xg, const void* gain) {
+    e.xg = reinterpret_cast<bf16*>(xg);
+    e.xg_gain = reinterpret_cast<const bf16*>(gain);
+    e.ss_part = ws.ss;
+    e.ss_ld = H / 128;
+    return e;
+  };
   EpiParams qkv_ep = make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos);
   qkv_ep.rope_cs = rope;
+  if (fuse && in_ready) {
+    FS_TRY(launch_rstd(ws.ss, H / 128, n, H, d->rms_eps, ws.rstd, st));
+    qkv_ep.row_rstd = ws.rstd;
+  } else {
+    FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
+  }
   FS_TRY(launch_linear(d, ws.xn, w->w_qkv, qkv_ep, n, 3 * A, H, st));
   FS_TRY(launch_attention(d, ws.qkv, ws.xn, n, st));
-  FS_TRY(launch_linear(d, ws.xn, w->w_o, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr), n, H, A,
-                       st));
-  FS_TRY(launch_rmsnorm_cast(x_out, w->g_ffn, ws.xn, n, H, d->rms_eps, d->dtype, st));
-  FS_TRY(launch_linear(d, ws.xn, w->w_1, make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr), n, F, H, st));
-  FS_TRY(launch_linear(d, ws.u, w->w_2, make_ep(d, FSDIT_EPI_RESIDUAL, w->b_2, x_out, H, x_out, nullptr), n, H, F,
-                       st));
+  // the FFN norm's operand goes to the qkv buffer (free after attention; the
+  // O projection still reads xn)
+  EpiParams o_ep = make_ep(d, FSDIT_EPI_RESIDUAL, w->b_o, x_out, H, x_in, nullptr);
+  if (fuse) o_ep = produce(o_ep, ws.qkv, w->g_ffn);
+  FS_TRY(launch_linear(d, ws.xn, w->w_o, o_ep, n, H, A, st));
+  EpiParams up_ep = make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr);
+  const void* up_a = ws.xn;
+  if (fuse) {
+    FS_TRY(launch_rstd(ws.ss, H / 128, n, H, d->rms_eps, ws.rstd, st));
+    up_ep.row_rstd = ws.rstd;
+    up_a = ws.qkv;
+  } else {
+    FS_TRY(launch_rmsnorm_cast(x_out, w->g_ffn, ws.xn, n, H, d->rms_eps, d->dtype, st));
+  }
+  FS_TRY(launch_linear(d, up_a, w->w_1, up_ep, n, F, H, st));
+  // the next block's attention-norm operand goes to xn (FFN-down reads u)
+  EpiParams down_ep = make_ep(d, FSDIT_EPI_RESIDUAL, w->b_2, x_out, H, x_out, nullptr);
+  if (fuse && g_next != nullptr) down_ep = produce(down_ep, ws.xn, g_next);
+  FS_TRY(launch_linear(d, ws.u, w->w_2, down_ep, n, H, F, st));
+  if (out_ready) *out_ready = fuse && g_next != nullptr;
   return FSDIT_OK;
 }
 
@@ -523,6 +573,7 @@ static size_t stack_carve(Carve& c, const fsdit_dims* d, const fsdit_io_weights*
     w.q8 = (uint8_t*)c.take((size_t)N * k8);
     w.sa = (float*)c.take((size_t)N * 4);
   }
+  carve_norm(c, d, N, w);
   *bw = w;
   return c.off;
 }
@@ -843,14 +894,21 @@ static fsdit_status stack_forward_impl(const fsdit_dims* dims, int n_layers, con
   const int n_grid = tok->grid_t * tok->grid_h * tok->grid_w;
   const int n_c = tok->keep_idx ? n_compressed(tok) : N;
   bool have_full_rope = false, have_comp_rope = false;
+  auto compressed = [&](int i) { return layer_compress[i] && tok->keep_idx != nullptr; };
+  // the next layer's attention norm is prepared by this layer's FFN-down
+  // epilogue when both run on the same rows
+  auto next_gain = [&](int i) -> const void* {
+    return i + 1 < n_layers && compressed(i + 1) == compressed(i) ? layers[i + 1].g_attn : nullptr;
+  };
+  bool ready = false;
   int l = 0;
   while (l < n_layers) {
-    if (!layer_compress[l] || tok->keep_idx == nullptr) {
+    if (!compressed(l)) {
       if (!have_full_rope) {
         FS_TRY(rope_table(dims, tok->pos_thw, N, bw.rope, st));
         have_full_rope = true;
       }
-      FS_TRY(block_body(dims, &layers[l], x, x, tok->pos_thw, bw.rope, N, bw, st));
+      FS_TRY(block_body(dims, &layers[l], x, x, tok->pos_thw, bw.rope, N, bw, st, ready, next_gain(l), &ready));
       ++l;
       continue;
     }
@@ -859,10 +917,13 @@ static fsdit_status stack_forward_impl(const fsdit_dims* dims, int n_layers, con
       FS_TRY(rope_table(dims, bw.posc, n_c, bw.rope_c, st));
       have_comp_rope = true;
     }
-    while (l < n_layers && layer_compress[l]) {
-      FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, bw.rope_c, n_c, bw, st));
+    ready = false;
+    while (l < n_layers && compressed(l)) {
+      FS_TRY(block_body(dims, &layers[l], bw.xc, bw.xc, bw.posc, bw.rope_c, n_c, bw, st, ready, next_gain(l),
+                        &ready));
       ++l;
     }
+    ready = false;
     FS_TRY(launch_broadcast(x, bw.xc, x, tok->keep_idx, tok->near_idx, tok->n_keep, tok->grid_t, tok->grid_h,
                             tok->grid_w, N, H, st));
   }

@@ -102,6 +102,17 @@ struct EpiParams {
   int up_rgb8;             // EPI_UNPATCH: 1 = write 8-bit codes (rgb8_code) instead of fp32 values
   float* split_part;       // pair GEMM tail cut: caller scratch for the partial accumulators
   int* split_cnt;          // (SPLIT_WS_BYTES) and its zeroed counters (SPLIT_CNT_BYTES), or null: no cut
+  // RMSNorm applied after the GEMM (bf16 tensor-core kernels, whole tiles):
+  // a consumer's operand is bf16(x * g) and row_rstd[row] = 1/rms(x) scales
+  // its accumulators before the bias; a RESIDUAL producer also writes that
+  // operand for the next norm, xg[row * ldo + col] = bf16(out * xg_gain[col]),
+  // and the sums of out^2 over each 128-column group p, ss_part[row * ss_ld + p]
+  // (N % 128 == 0).
+  const float* row_rstd = nullptr;
+  bf16* xg = nullptr;
+  const bf16* xg_gain = nullptr;
+  float* ss_part = nullptr;
+  int ss_ld = 0;
 };
 
 // Scratch of the pair GEMM's tail cut: 128 units of 256 KB fp32 partials and
@@ -140,12 +151,18 @@ __device__ __forceinline__ long long unpatch_offset(const EpiParams& p, int row,
 
 // Apply the epilogue to `cnt` consecutive columns [col, col+cnt) of one row.
 // v[] holds the fp32 accumulators; cnt is even and col is even.
+// Returns the sum of squares of the RESIDUAL outputs when p.xg is set, else 0.
 template <typename TW, int CNT>
-__device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int col, float* v) {
+__device__ __forceinline__ float epilogue_row(const EpiParams& p, int row, int col, float* v) {
   if (p.col_scale != nullptr) {
     const float rs = p.row_scale[row];
 #pragma unroll
     for (int i = 0; i < CNT; ++i) v[i] *= rs * p.col_scale[col + i];
+  }
+  if (p.row_rstd != nullptr) {
+    const float rs = p.row_rstd[row];
+#pragma unroll
+    for (int i = 0; i < CNT; ++i) v[i] *= rs;
   }
   const TW* bias = reinterpret_cast<const TW*>(p.bias);
 #pragma unroll
@@ -186,17 +203,27 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
   } else if (p.epi == FSDIT_EPI_RESIDUAL) {
     const float* r = p.resid + (size_t)row * p.ldr + col;
     float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
+    float ss = 0.0f;
     if constexpr (CNT % 4 == 0) {
 #pragma unroll
       for (int i = 0; i < CNT; i += 4) {
         float4 rv = *reinterpret_cast<const float4*>(r + i);
         float4 ov = make_float4(rv.x + v[i], rv.y + v[i + 1], rv.z + v[i + 2], rv.w + v[i + 3]);
         *reinterpret_cast<float4*>(o + i) = ov;
+        if (p.xg != nullptr) {
+          const bf16* g = p.xg_gain + col + i;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(ov.x * __bfloat162float(g[0]), ov.y * __bfloat162float(g[1]));
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(ov.z * __bfloat162float(g[2]), ov.w * __bfloat162float(g[3]));
+          *reinterpret_cast<uint2*>(p.xg + (size_t)row * p.ldo + col + i) =
+              make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+          ss += ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w;
+        }
       }
     } else {
 #pragma unroll
       for (int i = 0; i < CNT; ++i) o[i] = r[i] + v[i];
     }
+    return ss;
   } else if (p.epi == FSDIT_EPI_BIAS_F32) {
     float* o = reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + col;
     if constexpr (CNT % 4 == 0) {
@@ -228,6 +255,7 @@ __device__ __forceinline__ void epilogue_row(const EpiParams& p, int row, int co
       for (int i = 0; i < CNT; ++i) o[i] = cvt_from_f32<TW>(v[i]);
     }
   }
+  return 0.0f;
 }
 
 // ------------------------------------------------ tensor-core GEMM epilogue
@@ -240,6 +268,7 @@ struct Epi32Pre {
   float4 extra[8];  // QKV_ROPE: 16 (cos, sin) pairs; RESIDUAL: 32 fp32 residual values
   float4 cscale[8]; // FP8 dequantization: 32 column scales (same for every row)
   float rscale;     //                     and this row's scale
+  float rrs;        // row_rstd[row] (RMSNorm after the GEMM)
 };
 
 // GELU (tanh form) with the hardware tanh approximation (relative error about
@@ -267,6 +296,7 @@ __device__ __forceinline__ void epi32_prefetch(const EpiParams& p, int row, int 
     for (int i = 0; i < 8; ++i) e.cscale[i] = __ldg(cs + i);
     e.rscale = __ldg(p.row_scale + row);
   }
+  if (p.row_rstd != nullptr) e.rrs = __ldg(p.row_rstd + row);
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
     if (col < p.rope_cols && p.rope_cs != nullptr) {
       const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (size_t)row * (p.head_dim >> 1) +
@@ -290,6 +320,10 @@ __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col
       v[4 * i + 2] *= e.rscale * e.cscale[i].z;
       v[4 * i + 3] *= e.rscale * e.cscale[i].w;
     }
+  }
+  if (p.row_rstd != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= e.rrs;
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -398,6 +432,8 @@ struct EpiTPre {
   float4 cscale;    // FP8 dequantization: the 4 column scales
   float rscale[8];  //                     and the row scale of each of the 8 rows
   float4 extra[8];  // QKV_ROPE: (cos, sin) of the lane's 2 pairs; RESIDUAL: 4 fp32 values; per row
+  float rrs[8];     // row_rstd of each of the 8 rows
+  uint2 gain;       // RESIDUAL producer: the 4 bf16 gains of the lane's columns
 };
 
 // Loads for columns [col, col + 32) (all inside the output) of the block whose
@@ -413,6 +449,11 @@ __device__ __forceinline__ void epiT_prefetch(const EpiParams& p, int row0, int 
 #pragma unroll
     for (int i = 0; i < 8; ++i) e.rscale[i] = r0 + 4 * i < M ? __ldg(p.row_scale + r0 + 4 * i) : 0.0f;
   }
+  if (p.row_rstd != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e.rrs[i] = r0 + 4 * i < M ? __ldg(p.row_rstd + r0 + 4 * i) : 0.0f;
+  }
+  if (p.xg != nullptr) e.gain = __ldg(reinterpret_cast<const uint2*>(p.xg_gain + cl));
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
     if (col < p.rope_cols && p.rope_cs != nullptr) {
       const int pair = (cl & (p.head_dim - 1)) >> 1;
@@ -430,10 +471,11 @@ __device__ __forceinline__ void epiT_prefetch(const EpiParams& p, int row0, int 
 }
 
 // The epilogue of the transposed block w (w[4i + j] = column cl + j of row
-// r0 + 4i): dequantization, bias, RoPE / GELU, then the residual add and the
-// store, or the unpatchify store.
+// r0 + 4i): dequantization or the RMSNorm row scale, bias, RoPE / GELU, then
+// the residual add and the store (with the next norm's operand and the lane's
+// sums of squares added to ssq[i] when p.xg is set), or the unpatchify store.
 __device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col, int M, int lane, float* w,
-                                           const EpiTPre& e) {
+                                           const EpiTPre& e, float* ssq = nullptr) {
   const int cl = col + 4 * (lane & 7);
   const int r0 = row0 + (lane >> 3);
   if (p.col_scale != nullptr) {
@@ -443,6 +485,15 @@ __device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col
       w[4 * i + 1] *= e.rscale[i] * e.cscale.y;
       w[4 * i + 2] *= e.rscale[i] * e.cscale.z;
       w[4 * i + 3] *= e.rscale[i] * e.cscale.w;
+    }
+  }
+  if (p.row_rstd != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[4 * i] *= e.rrs[i];
+      w[4 * i + 1] *= e.rrs[i];
+      w[4 * i + 2] *= e.rrs[i];
+      w[4 * i + 3] *= e.rrs[i];
     }
   }
   {
@@ -546,8 +597,17 @@ __device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col
     const float* x = w + 4 * i;
     if (p.epi == FSDIT_EPI_RESIDUAL) {
       const float4 r = e.extra[i];
-      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) =
-          make_float4(r.x + x[0], r.y + x[1], r.z + x[2], r.w + x[3]);
+      const float4 o = make_float4(r.x + x[0], r.y + x[1], r.z + x[2], r.w + x[3]);
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) = o;
+      if (p.xg != nullptr) {
+        const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e.gain.x));
+        const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e.gain.y));
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(o.x * g01.x, o.y * g01.y);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(o.z * g23.x, o.w * g23.y);
+        *reinterpret_cast<uint2*>(p.xg + (size_t)row * p.ldo + cl) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+        ssq[i] += o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+      }
     } else if (p.epi == FSDIT_EPI_BIAS_F32) {
       *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)row * p.ldo + cl) =
           make_float4(x[0], x[1], x[2], x[3]);
@@ -570,7 +630,7 @@ namespace fsdit {
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
   PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_QUANT,
-  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_GRID_POS, PC_PIXEL_HEAD, PC_COUNT
+  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_GRID_POS, PC_PIXEL_HEAD, PC_RSTD, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);

@@ -63,6 +63,7 @@ static size_t decoder_carve(Carve& c, const fsdit_dims* d, int N, float** x, int
   *x = (float*)c.take((size_t)N * d->hidden * 4);
   *pos = (int32_t*)c.take((size_t)N * 3 * 4);
   *ws = carve_block(c, d, N, N, false);
+  carve_norm(c, d, N, *ws);
   return c.off;
 }
 
@@ -122,7 +123,10 @@ fsdit_status fsdit_decoder_forward(const fsdit_dims* dims, int n_layers, const f
   FS_TRY(launch_embed(dims->dtype, x, Hd, 0, N, 1, latents, io->c_lat, io->w_in, io->b_in, nullptr, nullptr,
                       nullptr, nullptr, nullptr, 0, 0, 0, st));
   FS_TRY(rope_table(dims, pos, N, ws.rope, st));
-  for (int l = 0; l < n_layers; ++l) FS_TRY(block_body(dims, &layers[l], x, x, pos, ws.rope, N, ws, st));
+  bool ready = false;  // each layer's FFN-down epilogue prepares the next layer's attention norm
+  for (int l = 0; l < n_layers; ++l)
+    FS_TRY(block_body(dims, &layers[l], x, x, pos, ws.rope, N, ws, st, ready,
+                      l + 1 < n_layers ? layers[l + 1].g_attn : nullptr, &ready));
   FS_TRY(launch_rmsnorm_cast(x, io->g_out, ws.xn, N, Hd, dims->rms_eps, dims->dtype, st));
   const int n_out = pixel_cols(io);
   EpiParams ep = make_ep(dims, EPI_UNPATCH, io->b_out, pixels, n_out, nullptr, nullptr);

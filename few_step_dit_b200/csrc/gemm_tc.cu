@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int row = mb * BM + q * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      float ss = 0.0f;  // RESIDUAL producer: sum of out^2 over the current 128-column group
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
@@ -175,7 +176,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int col = nb * BN + c * 32;
         if (row < args.M && col < args.N) {
           if (col + 32 <= args.N) {
-            epilogue_row<bf16, 32>(args.ep, row, col, v);
+            ss += epilogue_row<bf16, 32>(args.ep, row, col, v);
+            if ((c & 3) == 3 && args.ep.ss_part != nullptr) {
+              args.ep.ss_part[(size_t)row * args.ep.ss_ld + (col >> 7)] = ss;
+              ss = 0.0f;
+            }
           } else {  // ragged last chunk (N % 32 != 0, N even)
 #pragma unroll
             for (int i = 0; i < 32; i += 2)
@@ -498,6 +503,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         continue;
       }
       const int row0 = row - lane;  // first row of this warp's 32 x 32 blocks
+      float ssq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // RESIDUAL producer: rows row0 + lane/8 + 4i
 #pragma unroll 1
       for (int c = c0; c < c0 + BN / 64; ++c) {
         const int col = nb * BN + c * 32;
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(t_row + (uint32_t)(c * 32), v);
           float w[32];
           warp_transpose32(epi_buf, v, w, lane);
-          epiT_apply(args.ep, row0, col, args.M, lane, w, pre);
+          epiT_apply(args.ep, row0, col, args.M, lane, w, pre, ssq);
         } else {
           tmem_ld32(t_row + (uint32_t)(c * 32), v);
           if (row_ok && col < args.N) {  // ragged last chunk (N % 32 != 0, N even)
@@ -516,6 +522,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = 0; i < 32; i += 2)
               if (col + i < args.N) epilogue_row<bf16, 2>(args.ep, row, col + i, v + i);
           }
+        }
+      }
+      if (args.ep.ss_part != nullptr) {
+        // the eight lanes of a row hold 4 columns each of the warp's 128: sum
+        // them (fixed order) and store the row's partial for this group
+        const int grp = (nb * BN + c0 * 32) >> 7;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float t = ssq[i];
+          t += __shfl_xor_sync(0xffffffffu, t, 1);
+          t += __shfl_xor_sync(0xffffffffu, t, 2);
+          t += __shfl_xor_sync(0xffffffffu, t, 4);
+          const int r = row0 + (lane >> 3) + 4 * i;
+          if ((lane & 7) == 0 && r < args.M) args.ep.ss_part[(size_t)r * args.ep.ss_ld + grp] = t;
         }
       }
       tc_fence_before();
