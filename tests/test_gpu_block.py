@@ -158,6 +158,19 @@ def test_bf16_stack_small_width():
     assert O.rel_l2(ga, ra) < 1e-2
 
 
+def test_bf16_stack_hidden_not_a_multiple_of_128():
+    # hidden 192: every norm of the stack runs as its own RMSNorm-cast pass
+    # (the norm-after-GEMM path needs hidden % 128 == 0); the 256-wide cases
+    # above take that path
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=192, heads=2, ffn=384,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=6,
+                 compress=(0, 1, 1, 1, 0, 0))
+    assert w.hidden % 128 != 0
+    (gv, ga), (rv, ra) = _stack_case(w, 6, [0.0, 0.2, 0.5])
+    assert O.rel_l2(gv, rv) < 1e-2
+    assert O.rel_l2(ga, ra) < 1e-2
+
+
 def test_sampler_cuda_graph_replay_equals_eager():
     # the whole few-step pass is launch-only host code, so it captures into one
     # CUDA graph; a replay must reproduce the eager result bit for bit
