@@ -322,14 +322,24 @@ def build_backbone(w, device, rank, proj_fp8=False):
     return bb, seq, inp
 
 
-def timed(fn, steps, stream):
+def timed(fn, steps, stream, per_step=None):
+    """Milliseconds for `steps` calls of fn on `stream` (events on both sides);
+    with a list `per_step`, also an event after every call (appended: ms of
+    each step), which adds no work between the steps."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if per_step is not None else []
     start.record(stream)
-    for _ in range(steps):
+    for i in range(steps):
         fn()
+        if marks:
+            marks[i].record(stream)
     end.record(stream)
     end.synchronize()
+    prev = start
+    for m in marks:
+        per_step.append(prev.elapsed_time(m))
+        prev = m
     return start.elapsed_time(end)
 
 
@@ -378,7 +388,8 @@ def run_fsdit(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(local_rank)
     R.barrier(world, device)
-    t_ms = timed(run, args.steps, stream)
+    step_ms = []
+    t_ms = timed(run, args.steps, stream, step_ms)
     R.barrier(world, device)
     clk = clocks.stop()
     api.device_error()
@@ -483,6 +494,11 @@ def run_fsdit(args, rank, world, local_rank):
         "e2e": {"value": R.weak_scaling_value(w.n_tokens * w.n_evals, world, e_ms / 1000.0), "unit": UNIT,
                 "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
+    if step_ms:
+        srt = sorted(step_ms)
+        line["step_ms"] = {"median": statistics.median(srt), "min": srt[0], "max": srt[-1],
+                           "note": "this rank's timed steps, one event after each replay (the pages' protocol: "
+                                   "median of repeated runs after warm-up)"}
     if prof_ms is not None:
         line["profiled_ms_per_step"] = prof_ms
     if full_ms is not None:
