@@ -17,7 +17,7 @@ static const char* kProfNames[PC_COUNT] = {"gemm_qkv_rope", "gemm_residual", "ge
                                            "broadcast",     "embed",         "time_mlp",  "heads",
                                            "euler",         "keep_map",  "rope_table", "history_gather",
                                            "quantize",      "gemm_fp8_qkv_rope", "gemm_fp8_residual",
-                                           "gemm_fp8_gelu", "grid_positions", "pixel_head", "rms_rstd"};
+                                           "gemm_fp8_gelu", "grid_positions", "pixel_head"};
 struct Prof {
   bool on = false;
   int used = 0;
@@ -65,7 +65,6 @@ fsdit_status launch_gather(const float* x, const int32_t* pos, float* xc, int32_
 fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const int32_t* keep_idx,
                               const int32_t* near_idx, int n_keep, int grid_t, int grid_h, int grid_w, int n_rows,
                               int hidden, cudaStream_t st);
-fsdit_status launch_rstd(const float* ss, int parts, int rows, int hidden, float eps, float* rstd, cudaStream_t st);
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,
                                  cudaStream_t st);
 fsdit_status launch_embed(int dtype, float* x, int hidden, int row0, int rows, int kind, const float* lat, int K,
@@ -258,13 +257,13 @@ struct BlockWs {  // every buffer null until a carve sets it
   uint8_t* q8 = nullptr;     // FP8 projections: [n, max(hidden, attn, ffn)] E4M3 operand
   float* sa = nullptr;       //                  [n] its row scales
   float* ss = nullptr;       // RMSNorm after the GEMM: [n, hidden/128] sums of squares per column group
-  float* rstd = nullptr;     //                         [n] 1/rms per row
 };
 
 // Blocks run back to back (stack, decoder) apply each RMSNorm after the GEMM
 // that consumes it: the residual epilogue before the norm writes bf16(x * g)
-// and per-group sums of squares, and the consuming GEMM scales its rows by
-// 1/rms.  bf16 tensor-core projections with hidden % 128 == 0 only.
+// and per-group sums of squares, and the consuming GEMM forms 1/rms of each
+// row from those sums and scales its accumulators by it.  bf16 tensor-core
+// projections with hidden % 128 == 0 only.
 static bool norm_after_gemm(const fsdit_dims* d) {
   return d->dtype == FSDIT_BF16 && !d->proj_fp8 && d->hidden % 128 == 0;
 }
@@ -272,7 +271,6 @@ static bool norm_after_gemm(const fsdit_dims* d) {
 static void carve_norm(Carve& c, const fsdit_dims* d, int n_rows, BlockWs& w) {
   if (!norm_after_gemm(d)) return;
   w.ss = (float*)c.take((size_t)n_rows * (d->hidden / 128) * 4);
-  w.rstd = (float*)c.take((size_t)n_rows * 4);
 }
 
 static BlockWs carve_block(Carve& c, const fsdit_dims* d, int n_rows, int n_c, bool compressed) {
@@ -350,7 +348,7 @@ static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w
   if (out_ready) *out_ready = false;
   if (d->proj_fp8) return block_body_fp8(d, w, x_in, x_out, pos, rope, n, ws, st);
   const int H = d->hidden, F = d->ffn, A = attn_dim(d);
-  const bool fuse = ws.ss != nullptr && ws.rstd != nullptr;
+  const bool fuse = ws.ss != nullptr;
   auto produce = [&](EpiParams e, void* xg, const void* gain) {
     e.xg = reinterpret_cast<bf16*>(xg);
     e.xg_gain = reinterpret_cast<const bf16*>(gain);
@@ -358,11 +356,16 @@ static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w
     e.ss_ld = H / 128;
     return e;
   };
+  auto consume = [&](EpiParams& e) {
+    e.norm_ss = ws.ss;
+    e.ss_ld = H / 128;
+    e.norm_h = H;
+    e.norm_eps = d->rms_eps;
+  };
   EpiParams qkv_ep = make_ep(d, FSDIT_EPI_QKV_ROPE, w->b_qkv, ws.qkv, 3 * A, nullptr, pos);
   qkv_ep.rope_cs = rope;
   if (fuse && in_ready) {
-    FS_TRY(launch_rstd(ws.ss, H / 128, n, H, d->rms_eps, ws.rstd, st));
-    qkv_ep.row_rstd = ws.rstd;
+    consume(qkv_ep);
   } else {
     FS_TRY(launch_rmsnorm_cast(x_in, w->g_attn, ws.xn, n, H, d->rms_eps, d->dtype, st));
   }
@@ -376,8 +379,7 @@ static fsdit_status block_body(const fsdit_dims* d, const fsdit_block_weights* w
   EpiParams up_ep = make_ep(d, FSDIT_EPI_GELU, w->b_1, ws.u, F, nullptr, nullptr);
   const void* up_a = ws.xn;
   if (fuse) {
-    FS_TRY(launch_rstd(ws.ss, H / 128, n, H, d->rms_eps, ws.rstd, st));
-    up_ep.row_rstd = ws.rstd;
+    consume(up_ep);
     up_a = ws.qkv;
   } else {
     FS_TRY(launch_rmsnorm_cast(x_out, w->g_ffn, ws.xn, n, H, d->rms_eps, d->dtype, st));

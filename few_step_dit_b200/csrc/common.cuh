@@ -102,17 +102,20 @@ struct EpiParams {
   int up_rgb8;             // EPI_UNPATCH: 1 = write 8-bit codes (rgb8_code) instead of fp32 values
   float* split_part;       // pair GEMM tail cut: caller scratch for the partial accumulators
   int* split_cnt;          // (SPLIT_WS_BYTES) and its zeroed counters (SPLIT_CNT_BYTES), or null: no cut
-  // RMSNorm applied after the GEMM (bf16 tensor-core kernels, whole tiles):
-  // a consumer's operand is bf16(x * g) and row_rstd[row] = 1/rms(x) scales
-  // its accumulators before the bias; a RESIDUAL producer also writes that
-  // operand for the next norm, xg[row * ldo + col] = bf16(out * xg_gain[col]),
-  // and the sums of out^2 over each 128-column group p, ss_part[row * ss_ld + p]
-  // (N % 128 == 0).
-  const float* row_rstd = nullptr;
+  // RMSNorm applied after the GEMM (bf16 tensor-core kernels): a RESIDUAL
+  // producer also writes the next norm's operand, xg[row * ldo + col] =
+  // bf16(out * xg_gain[col]), and the sums of out^2 over each 128-column
+  // group p, ss_part[row * ss_ld + p] (N % 128 == 0, whole tiles); a consumer
+  // (operand bf16(x * g)) with norm_ss set scales its accumulators before the
+  // bias by 1/rms(x) = rsqrt(sum of the norm_h / 128 groups of
+  // norm_ss[row * ss_ld ..] in group order / norm_h + norm_eps).
   bf16* xg = nullptr;
   const bf16* xg_gain = nullptr;
   float* ss_part = nullptr;
   int ss_ld = 0;
+  const float* norm_ss = nullptr;
+  int norm_h = 0;
+  float norm_eps = 0.0f;
 };
 
 // Scratch of the pair GEMM's tail cut: 128 units of 256 KB fp32 partials and
@@ -151,6 +154,24 @@ __device__ __forceinline__ long long unpatch_offset(const EpiParams& p, int row,
 
 // Apply the epilogue to `cnt` consecutive columns [col, col+cnt) of one row.
 // v[] holds the fp32 accumulators; cnt is even and col is even.
+// 1/rms of `row` from its producer's per-group sums of squares (the same
+// order in every tile and kernel, so every tile of a row scales it alike).
+__device__ __forceinline__ float norm_rstd(const EpiParams& p, int row) {
+  const float* ss = p.norm_ss + (size_t)row * p.ss_ld;
+  const int groups = p.norm_h >> 7;
+  float t = 0.0f;
+  int g = 0;
+  for (; g + 8 <= groups; g += 8) {  // eight loads in flight, added in order
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = __ldg(ss + g + k);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += a[k];
+  }
+  for (; g < groups; ++g) t += __ldg(ss + g);
+  return rsqrtf(t / (float)p.norm_h + p.norm_eps);
+}
+
 // Returns the sum of squares of the RESIDUAL outputs when p.xg is set, else 0.
 template <typename TW, int CNT>
 __device__ __forceinline__ float epilogue_row(const EpiParams& p, int row, int col, float* v) {
@@ -159,8 +180,8 @@ __device__ __forceinline__ float epilogue_row(const EpiParams& p, int row, int c
 #pragma unroll
     for (int i = 0; i < CNT; ++i) v[i] *= rs * p.col_scale[col + i];
   }
-  if (p.row_rstd != nullptr) {
-    const float rs = p.row_rstd[row];
+  if (p.norm_ss != nullptr) {
+    const float rs = norm_rstd(p, row);
 #pragma unroll
     for (int i = 0; i < CNT; ++i) v[i] *= rs;
   }
@@ -268,7 +289,7 @@ struct Epi32Pre {
   float4 extra[8];  // QKV_ROPE: 16 (cos, sin) pairs; RESIDUAL: 32 fp32 residual values
   float4 cscale[8]; // FP8 dequantization: 32 column scales (same for every row)
   float rscale;     //                     and this row's scale
-  float rrs;        // row_rstd[row] (RMSNorm after the GEMM)
+  float rrs;        // 1/rms of the row (RMSNorm after the GEMM)
 };
 
 // GELU (tanh form) with the hardware tanh approximation (relative error about
@@ -296,7 +317,7 @@ __device__ __forceinline__ void epi32_prefetch(const EpiParams& p, int row, int 
     for (int i = 0; i < 8; ++i) e.cscale[i] = __ldg(cs + i);
     e.rscale = __ldg(p.row_scale + row);
   }
-  if (p.row_rstd != nullptr) e.rrs = __ldg(p.row_rstd + row);
+  if (p.norm_ss != nullptr) e.rrs = norm_rstd(p, row);
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
     if (col < p.rope_cols && p.rope_cs != nullptr) {
       const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (size_t)row * (p.head_dim >> 1) +
@@ -321,7 +342,7 @@ __device__ __forceinline__ void epi32_apply(const EpiParams& p, int row, int col
       v[4 * i + 3] *= e.rscale * e.cscale[i].w;
     }
   }
-  if (p.row_rstd != nullptr) {
+  if (p.norm_ss != nullptr) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= e.rrs;
   }
@@ -432,15 +453,17 @@ struct EpiTPre {
   float4 cscale;    // FP8 dequantization: the 4 column scales
   float rscale[8];  //                     and the row scale of each of the 8 rows
   float4 extra[8];  // QKV_ROPE: (cos, sin) of the lane's 2 pairs; RESIDUAL: 4 fp32 values; per row
-  float rrs[8];     // row_rstd of each of the 8 rows
+  float rrs[8];     // 1/rms of each of the 8 rows
   uint2 gain;       // RESIDUAL producer: the 4 bf16 gains of the lane's columns
 };
 
 // Loads for columns [col, col + 32) (all inside the output) of the block whose
 // first row is row0; rows at or past M are skipped.  Alignment as for
 // epi32_prefetch.
+// lane_rstd: with p.norm_ss, 1/rms of row row0 + lane (norm_rstd), computed
+// once per tile by the caller.
 __device__ __forceinline__ void epiT_prefetch(const EpiParams& p, int row0, int col, int M, int lane,
-                                              EpiTPre& e) {
+                                              EpiTPre& e, float lane_rstd = 0.0f) {
   const int cl = col + 4 * (lane & 7);
   const int r0 = row0 + (lane >> 3);
   e.bias = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(p.bias) + cl));
@@ -449,9 +472,9 @@ __device__ __forceinline__ void epiT_prefetch(const EpiParams& p, int row0, int 
 #pragma unroll
     for (int i = 0; i < 8; ++i) e.rscale[i] = r0 + 4 * i < M ? __ldg(p.row_scale + r0 + 4 * i) : 0.0f;
   }
-  if (p.row_rstd != nullptr) {
+  if (p.norm_ss != nullptr) {  // lane k holds row row0 + k's (whole warp, converged)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) e.rrs[i] = r0 + 4 * i < M ? __ldg(p.row_rstd + r0 + 4 * i) : 0.0f;
+    for (int i = 0; i < 8; ++i) e.rrs[i] = __shfl_sync(0xffffffffu, lane_rstd, (lane >> 3) + 4 * i);
   }
   if (p.xg != nullptr) e.gain = __ldg(reinterpret_cast<const uint2*>(p.xg_gain + cl));
   if (p.epi == FSDIT_EPI_QKV_ROPE) {
@@ -487,7 +510,7 @@ __device__ __forceinline__ void epiT_apply(const EpiParams& p, int row0, int col
       w[4 * i + 3] *= e.rscale[i] * e.cscale.w;
     }
   }
-  if (p.row_rstd != nullptr) {
+  if (p.norm_ss != nullptr) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       w[4 * i] *= e.rrs[i];
@@ -630,7 +653,7 @@ namespace fsdit {
 enum ProfClass {
   PC_GEMM_QKV, PC_GEMM_RESID, PC_GEMM_GELU, PC_GEMM_BIAS_F32, PC_GEMM_BIAS, PC_ATTN, PC_NORM,
   PC_GATHER, PC_BCAST, PC_EMBED, PC_TIMEMLP, PC_HEADS, PC_EULER, PC_KEEPMAP, PC_ROPE, PC_HISTORY, PC_QUANT,
-  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_GRID_POS, PC_PIXEL_HEAD, PC_RSTD, PC_COUNT
+  PC_GEMM_FP8_QKV, PC_GEMM_FP8_RESID, PC_GEMM_FP8_GELU, PC_GRID_POS, PC_PIXEL_HEAD, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, int kernels, double flops, double bytes, cudaStream_t st);

@@ -196,25 +196,6 @@ __global__ void __launch_bounds__(256) rmsnorm_cast_kernel(const float* __restri
   }
 }
 
-// rstd[r] = 1 / sqrt(mean(x_r^2) + eps) from the row's sums of squares over
-// its `parts` column groups (written by a RESIDUAL GEMM epilogue).  One warp
-// per row: lane i adds groups i, i + 32, ..., then a fixed butterfly sums the
-// lanes, so every run adds in the same order.  With the operand bf16(x * g)
-// the GEMM that follows applies rstd to its accumulators: RMSNorm with the
-// scale moved after the product.
-__global__ void __launch_bounds__(256) rstd_kernel(const float* __restrict__ ss, int parts, int rows, int hidden,
-                                                   float eps, float* __restrict__ rstd) {
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const float* p = ss + (size_t)r * parts;
-  float s = 0.f;
-  for (int i = lane; i < parts; i += 32) s += p[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) rstd[r] = rsqrtf(s / (float)hidden + eps);
-}
-
 // ---------------------------------------------------------------- RoPE table
 // cs[r][j] = (cos, sin) of the angle of pair j of a head for row r; the QKV
 // epilogue reads it instead of evaluating sincos per element.  Positions are
@@ -501,13 +482,6 @@ fsdit_status launch_broadcast(const float* x, const float* yc, float* out, const
   broadcast_kernel<<<grid_for_rows(n_blocks, 8), 256, 0, st>>>(x, yc, out, keep_idx, near_idx, n_keep, grid_h,
                                                                grid_w, n_grid, n_rows, hidden);
   return cuda_check(cudaGetLastError(), "broadcast_kernel");
-}
-
-fsdit_status launch_rstd(const float* ss, int parts, int rows, int hidden, float eps, float* rstd, cudaStream_t st) {
-  if (rows <= 0) return FSDIT_OK;
-  ProfScope ps(PC_RSTD, 1, 0.0, (double)rows * (parts + 1) * 4.0, st);
-  rstd_kernel<<<(rows + 7) / 8, 256, 0, st>>>(ss, parts, rows, hidden, eps, rstd);
-  return cuda_check(cudaGetLastError(), "rstd_kernel");
 }
 
 fsdit_status launch_rmsnorm_cast(const float* x, const void* g, void* xn, int rows, int hidden, float eps, int dtype,

@@ -489,14 +489,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       int mb, nb;
       gemm::tile_coords(tile, args, mb, nb);
+      const int row = mb * BM + (int)rank * HM + q * 32 + lane;
+      const bool row_ok = row < args.M;
+      // RMSNorm consumer: 1/rms of this lane's row, read while the tile's
+      // accumulators are still being computed
+      const float lane_rstd = !SPLIT && args.ep.norm_ss != nullptr && row_ok ? norm_rstd(args.ep, row) : 0.0f;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(TFULL(buf), aph, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int row = mb * BM + (int)rank * HM + q * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-      const bool row_ok = row < args.M;
       if constexpr (SPLIT) {
         split_unit_epilogue(args, t_row, slot, sp, region, row, row_ok, nb, c0, lane,
                             rank == 0 ? TEMPTY(buf) : tempty0 + 8u * (uint32_t)buf, rank == 0);
@@ -510,7 +513,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[32];
         if (col + 32 <= args.N) {  // warp-uniform: the block's columns are all inside
           EpiTPre pre;
-          epiT_prefetch(args.ep, row0, col, args.M, lane, pre);
+          epiT_prefetch(args.ep, row0, col, args.M, lane, pre, lane_rstd);
           tmem_ld32(t_row + (uint32_t)(c * 32), v);
           float w[32];
           warp_transpose32(epi_buf, v, w, lane);

@@ -367,10 +367,10 @@ FSDIT_API fsdit_status dit_block_forward(const fsdit_dims* dims, const fsdit_blo
  * arithmetic), final RMSNorm and the video/audio velocity heads.  With bf16
  * dense projections and hidden % 128 == 0, a norm that follows a residual
  * projection on the same rows is applied after the GEMM that consumes it:
- * the residual epilogue writes bf16(x * g) and per-128-column sums of x^2, a
- * small kernel turns those into 1/rms per row, and the consuming GEMM scales
- * its accumulators by it (the same RMSNorm in exact arithmetic; in bf16 the
- * operand is rounded before the row scale instead of after it).
+ * the residual epilogue writes bf16(x * g) and per-128-column sums of x^2,
+ * and the consuming GEMM's epilogue forms 1/rms of each row from those sums
+ * and scales its accumulators by it (the same RMSNorm in exact arithmetic; in
+ * bf16 the operand is rounded before the row scale instead of after it).
  *   time_table (host) float [n_times], n_times <= 8
  *   video_lat float32 [n_vrows, c_video], audio_lat float32 [n_audio, c_audio],
  *   text_emb `dtype` [n_text, c_text]                      (device, inputs)
