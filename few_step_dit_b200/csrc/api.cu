@@ -264,8 +264,9 @@ struct BlockWs {  // every buffer null until a carve sets it
 // and per-group sums of squares, and the consuming GEMM forms 1/rms of each
 // row from those sums and scales its accumulators by it.  bf16 tensor-core
 // projections with hidden % 128 == 0 only.
+static int g_norm_after_gemm = 1;  // fsdit_set_norm_after_gemm
 static bool norm_after_gemm(const fsdit_dims* d) {
-  return d->dtype == FSDIT_BF16 && !d->proj_fp8 && d->hidden % 128 == 0;
+  return g_norm_after_gemm != 0 && d->dtype == FSDIT_BF16 && !d->proj_fp8 && d->hidden % 128 == 0;
 }
 
 static void carve_norm(Carve& c, const fsdit_dims* d, int n_rows, BlockWs& w) {
@@ -801,6 +802,17 @@ fsdit_status fsdit_linear_fp8_ws(const fsdit_dims* dims, const uint8_t* qa, cons
   FS_TRY(attach_scratch(ep, scratch, scratch_bytes, (cudaStream_t)stream));
   return launch_linear_fp8(dims, qa, qw, ep, M, N, K, (cudaStream_t)stream);
 }
+
+fsdit_status fsdit_set_norm_after_gemm(int on) {
+  if (on != 0 && on != 1) {
+    set_error("set_norm_after_gemm: on must be 0 or 1, got %d", on);
+    return FSDIT_E_SHAPE;
+  }
+  g_norm_after_gemm = on;
+  return FSDIT_OK;
+}
+
+int fsdit_norm_after_gemm(void) { return g_norm_after_gemm; }
 
 fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, void* out, int n, fsdit_stream_t stream) {
   FS_TRY(check_dims(dims));

@@ -105,6 +105,8 @@ _SIGS = {
     "fsdit_attention": (_I, [C.POINTER(Dims), _P, _P, _I, _P]),
     "fsdit_set_attention_pair_min_rows": (_I, [_I]),
     "fsdit_attention_pair_min_rows": (_I, []),
+    "fsdit_set_norm_after_gemm": (_I, [_I]),
+    "fsdit_norm_after_gemm": (_I, []),
     "dit_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), C.POINTER(Tokens), _P, _P,
                                _P, C.c_size_t, _P]),
     "dit_block_forward_noalloc": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), C.POINTER(Tokens),

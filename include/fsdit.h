@@ -340,7 +340,7 @@ FSDIT_API fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, 
                              fsdit_stream_t stream);
 
 /* Attention kernel choice (bf16).  Sequences of at least `rows` rows run on
- * the CTA-pair kernel (clusters of two CTAs, 512 queries per cluster, each
+ * the CTA-pair kernel (clusters of two CTAs, 256 queries per cluster, each
  * CTA staging half of every key and value block); shorter ones on the
  * single-CTA kernel (256 queries per CTA).  Both compute the same attention;
  * the threshold is a tuning knob for the whole process (not thread-safe
@@ -348,6 +348,17 @@ FSDIT_API fsdit_status fsdit_attention(const fsdit_dims* dims, const void* qkv, 
  * current value.  Errors: FSDIT_E_SHAPE for rows < 1. */
 FSDIT_API fsdit_status fsdit_set_attention_pair_min_rows(int rows);
 FSDIT_API int fsdit_attention_pair_min_rows(void);
+
+/* RMSNorm placement in stacks and the decoder (dit_stack_forward and what
+ * calls it, fsdit_decoder_forward): on = 1 (the default) applies a norm that
+ * follows a residual projection after the GEMM that consumes it (see
+ * dit_stack_forward); on = 0 runs every norm as its own fsdit_rmsnorm_cast
+ * pass.  The same RMSNorm either way, rounded in a different order.  A
+ * process-wide switch (not thread-safe against concurrent launches); query
+ * workspace sizes after setting it.  fsdit_norm_after_gemm returns the
+ * current value.  Errors: FSDIT_E_SHAPE unless on is 0 or 1. */
+FSDIT_API fsdit_status fsdit_set_norm_after_gemm(int on);
+FSDIT_API int fsdit_norm_after_gemm(void);
 
 /* One DiT block.  x_in, x_out float32 [n_tokens, hidden] (device);
  * x_out may equal x_in.  With tok->keep_idx != NULL the block is the Flash

@@ -1,5 +1,5 @@
-"""The CTA-pair attention kernel (clusters of two CTAs, 512 queries per
-cluster, P staged in shared memory) against the oracle's fp64 softmax and
+"""The CTA-pair attention kernel (clusters of two CTAs, 256 queries per
+cluster, Q and P in tensor memory) against the oracle's fp64 softmax and
 against the single-CTA kernel, on ragged and full-size sequences and on the
 score distributions that drive the online softmax ([tokendh] backbone
 section: one joint sequence of text, video and audio tokens, no mask).
@@ -63,8 +63,8 @@ def test_threshold_knob_rejects_nonpositive(_pair_everywhere):
 
 @pytest.mark.parametrize("n", [1, 64, 128, 129, 300, 511, 512, 513, 1000, 1300, 3668])
 def test_pair_attention_matches_oracle_and_single_cta_kernel(_pair_everywhere, n):
-    # one cluster covers 512 queries (two 256-row pair tiles); 513 and 1300
-    # leave ragged clusters, 129 a ragged key block split across the pair
+    # one cluster covers 256 queries (a 128-row tile per CTA); 300, 513 and
+    # 1300 leave ragged clusters, 129 a ragged key block split across the pair
     heads = 2
     A = heads * 128
     g = torch.Generator().manual_seed(n)

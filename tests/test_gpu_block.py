@@ -171,6 +171,32 @@ def test_bf16_stack_hidden_not_a_multiple_of_128():
     assert O.rel_l2(ga, ra) < 1e-2
 
 
+def test_norm_after_gemm_against_separate_norm_passes():
+    # the same 8-layer bf16 stack (hidden 256) with every norm as its own
+    # RMSNorm-cast pass (switch off) and with the norms that follow a residual
+    # projection applied after their consuming GEMM (the default): both within
+    # the bf16 bound of the oracle, and within a few bf16 roundings of each
+    # other (the operand is rounded before the row scale instead of after it)
+    fs = L.load()
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=256, heads=2, ffn=512,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=8,
+                 compress=(0, 0, 1, 1, 1, 1, 0, 0))
+    assert fs.fsdit_norm_after_gemm() == 1
+    (gv, ga), (rv, ra) = _stack_case(w, 8, [0.0, 0.2, 0.5])
+    assert fs.fsdit_set_norm_after_gemm(0) == 0
+    try:
+        (sv, sa), _ = _stack_case(w, 8, [0.0, 0.2, 0.5])
+    finally:
+        assert fs.fsdit_set_norm_after_gemm(1) == 0
+    for got in ((gv, ga), (sv, sa)):
+        assert O.rel_l2(got[0], rv) < 1e-2
+        assert O.rel_l2(got[1], ra) < 1e-2
+    assert O.rel_l2(gv, sv) < 5e-3
+    assert O.rel_l2(ga, sa) < 5e-3
+    assert not np.array_equal(gv, sv)  # the switch changed the path
+    assert fs.fsdit_set_norm_after_gemm(2) == -2
+
+
 def test_sampler_cuda_graph_replay_equals_eager():
     # the whole few-step pass is launch-only host code, so it captures into one
     # CUDA graph; a replay must reproduce the eager result bit for bit
