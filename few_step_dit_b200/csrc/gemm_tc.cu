@@ -527,9 +527,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (args.ep.ss_part != nullptr) {
+      if (args.ep.ss_part != nullptr && nb * BN + c0 * 32 < args.N) {
         // the eight lanes of a row hold 4 columns each of the warp's 128: sum
-        // them (fixed order) and store the row's partial for this group
+        // them (fixed order) and store the row's partial for this group (a
+        // warp whose columns lie past N -- the last tile of an N that is an
+        // odd multiple of 128 -- has no group)
         const int grp = (nb * BN + c0 * 32) >> 7;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {

@@ -197,6 +197,18 @@ def test_norm_after_gemm_against_separate_norm_passes():
     assert fs.fsdit_set_norm_after_gemm(2) == -2
 
 
+def test_bf16_stack_hidden_an_odd_multiple_of_128():
+    # hidden 384: the residual GEMMs' last 256-column tile is half outside
+    # the output, so its second column half has no sum-of-squares group
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=384, heads=2, ffn=512,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=6,
+                 compress=(0, 1, 1, 1, 0, 0))
+    assert w.hidden % 128 == 0 and w.hidden % 256 != 0
+    (gv, ga), (rv, ra) = _stack_case(w, 6, [0.0, 0.2, 0.5])
+    assert O.rel_l2(gv, rv) < 1e-2
+    assert O.rel_l2(ga, ra) < 1e-2
+
+
 def test_sampler_cuda_graph_replay_equals_eager():
     # the whole few-step pass is launch-only host code, so it captures into one
     # CUDA graph; a replay must reproduce the eager result bit for bit
