@@ -209,6 +209,19 @@ def test_bf16_stack_hidden_an_odd_multiple_of_128():
     assert O.rel_l2(ga, ra) < 1e-2
 
 
+@pytest.mark.parametrize("hidden,heads,ffn", [(128, 1, 256), (256, 3, 384), (512, 2, 640), (640, 1, 1024),
+                                              (768, 4, 512)])
+def test_bf16_stack_widths(hidden, heads, ffn):
+    # hidden and attention widths that differ, hidden an even or odd multiple
+    # of 128 (the norm-after-GEMM path), FFN widths that leave ragged tiles
+    w = S.scaled(S.WORKLOADS["flash_backbone_6x34x60"], hidden=hidden, heads=heads, ffn=ffn,
+                 grid=(2, 9, 10), n_text=16, n_audio=8, n_layers=5,
+                 compress=(0, 1, 1, 0, 0))
+    (gv, ga), (rv, ra) = _stack_case(w, 5, [0.0, 0.2, 0.5])
+    assert O.rel_l2(gv, rv) < 1e-2
+    assert O.rel_l2(ga, ra) < 1e-2
+
+
 def test_sampler_cuda_graph_replay_equals_eager():
     # the whole few-step pass is launch-only host code, so it captures into one
     # CUDA graph; a replay must reproduce the eager result bit for bit
