@@ -116,6 +116,37 @@ def test_sampler_with_empty_modalities(n_text, n_audio):
         assert O.rel_l2(al.double().cpu().numpy(), ra) < 1e-5
 
 
+@pytest.mark.parametrize("grid,n_text,n_audio", [((1, 1, 1), 16, 8), ((3, 2, 2), 5, 3), ((1, 2, 7), 0, 1),
+                                                 ((2, 9, 10), 0, 0)])
+def test_bf16_sampler_on_tiny_sequences(grid, n_text, n_audio):
+    # bf16 at hidden 256 (the stack applies each norm after its consuming
+    # GEMM) on sequences of 13 to 180 rows: the projections run on the
+    # single-CTA GEMM (M <= 128) or on partly filled pair tiles
+    w = _tiny(grid=grid, n_text=n_text, n_audio=n_audio, n_layers=4, compress=(0, 1, 1, 0), dtype="bf16",
+              video_clock=S.WORKLOADS["flash_backbone_6x34x60"].video_clock,
+              audio_clock=S.WORKLOADS["flash_backbone_6x34x60"].audio_clock)
+    layers, io = S.make_weights(w)
+    inp = S.make_inputs(w)
+    tags = S.pack_tokens(w)
+    seq = api.Sequence.from_workload(w, tags, DEV)
+    bb = api.Backbone(api.dims_of(w), [api.BlockWeights({k: v.to(DEV) for k, v in l.items()}) for l in layers],
+                      api.IOWeights({k: v.to(DEV) for k, v in io.items()}), w.compress)
+    vl, al = inp["video_lat"].to(DEV).clone(), inp["audio_lat"].to(DEV).clone()
+    bb.sample(seq, w.video_clock, w.audio_clock, vl, inp["text_emb"].to(DEV), al)
+    torch.cuda.synchronize()
+    tok = dict(tags)
+    tok["keep_idx"], tok["near_idx"] = O.keep_map(*w.grid)
+    rv, ra = O.flow_sample([S.to_numpy64(l) for l in layers], w.compress, S.to_numpy64(io), tok, w.video_clock,
+                           w.audio_clock, inp["video_lat"].double().numpy(), inp["text_emb"].double().numpy(),
+                           inp["audio_lat"].double().numpy(), w.heads, w.head_dim)
+    v0 = inp["video_lat"].double().numpy()
+    got = vl.double().cpu().numpy()
+    assert O.rel_l2(got, rv) < 1e-2
+    assert O.rel_l2(got - v0, rv - v0) < 1e-2
+    if n_audio:
+        assert O.rel_l2(al.double().cpu().numpy(), ra) < 1e-2
+
+
 def test_smallest_long_video_chunks():
     # T = 2: each later chunk is one boundary latent and one new latent
     w = _tiny(grid=(2, 4, 5), n_layers=2, compress=(1, 0))
